@@ -1,0 +1,158 @@
+"""Gated DeltaNet token mixer forward pass for NVIDIA B200 (sm_100a).
+
+A thin ctypes binding over ``libgdn.so`` (declared in ``include/gdn.h``):
+argument marshalling only -- every step of the computation runs in the CUDA
+kernels of the library. PyTorch provides device memory and streams. There is
+no CPU fallback: if the library is missing the import of an op fails loudly.
+
+    o, state_out = prefill(q, k, v, g, beta, state_in=None, cu_seqlens=None)
+    o = decode(q, k, v, g, beta, state)          # state updated in place
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+__all__ = ["prefill", "decode", "prefill_workspace_bytes", "device_error", "GdnError",
+           "lib", "library_path", "GDN_BF16", "GDN_F32"]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_PKG, "libgdn.so")
+
+GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_DEVICE_TIMEOUT = range(5)
+GDN_BF16, GDN_F32 = 0, 1
+STATUS_NAMES = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED",
+                3: "GDN_ERR_CUDA", 4: "GDN_ERR_DEVICE_TIMEOUT"}
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+_lock = threading.Lock()
+_lib = None
+
+_vp, _fp, _i32p = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p
+_i, _i64, _f, _sz = ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+
+SIGNATURES = {
+    "gdn_version": (_i, []),
+    "gdn_last_error": (ctypes.c_char_p, []),
+    "gdn_prefill_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
+    "gdn_prefill": (_i, [_vp, _vp, _vp, _fp, _fp, _fp, _i32p, _i, _i64, _i, _i, _i, _i, _f, _i, _i,
+                         _vp, _fp, _vp, _sz, _vp]),
+    "gdn_decode": (_i, [_vp, _vp, _vp, _fp, _fp, _fp, _i, _i, _i, _i, _i, _f, _i, _vp, _vp]),
+    "gdn_device_error": (_i, [_vp]),
+}
+
+
+def lib():
+    """Load libgdn.so (built in-tree); raises if it is missing."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(library_path):
+                raise ImportError(
+                    f"{library_path} is missing: build it with "
+                    "`python -m gated_deltanet_linear_21_b200.build` (there is no CPU fallback)")
+            handle = ctypes.CDLL(library_path)
+            for name, (res, args) in SIGNATURES.items():
+                fn = getattr(handle, name)
+                fn.restype, fn.argtypes = res, args
+            _lib = handle
+    return _lib
+
+
+def _check(status: int):
+    if status != GDN_OK:
+        raise GdnError(status, lib().gdn_last_error().decode())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return GDN_BF16
+    if t.dtype == torch.float32:
+        return GDN_F32
+    raise TypeError(f"q, k, v must be bf16 or fp32, got {t.dtype}")
+
+
+def _dev(t, name, dtype=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t
+
+
+def _stream_handle(stream) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def prefill_workspace_bytes(n_seqs, Hv, dk, dv, dtype=torch.bfloat16) -> int:
+    code = GDN_BF16 if dtype == torch.bfloat16 else GDN_F32
+    return int(lib().gdn_prefill_workspace_bytes(n_seqs, Hv, dk, dv, code))
+
+
+def prefill(q, k, v, g, beta, state_in=None, cu_seqlens=None, *, scale=None, chunk=0,
+            o=None, state_out=None, workspace=None, stream=None):
+    """Chunked prefill over packed sequences.
+
+    q, k [T, Hqk, dk]; v [T, Hv, dv] (bf16 or fp32, same dtype); g, beta [T, Hv]
+    fp32; state_in [N, Hv, dv, dk] fp32 or None; cu_seqlens [N+1] int32 (None =
+    one sequence of T tokens). Returns (o [T, Hv, dv], state_out [N, Hv, dv, dk]).
+    """
+    _dev(q, "q"); _dev(k, "k", q.dtype); _dev(v, "v", q.dtype)
+    _dev(g, "g", torch.float32); _dev(beta, "beta", torch.float32)
+    T, Hqk, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[2]
+    if cu_seqlens is None:
+        cu_seqlens = torch.tensor([0, T], dtype=torch.int32, device=q.device)
+    _dev(cu_seqlens, "cu_seqlens", torch.int32)
+    N = cu_seqlens.numel() - 1
+    if state_in is not None:
+        _dev(state_in, "state_in", torch.float32)
+    if o is None:
+        o = torch.empty(T, Hv, dv, dtype=q.dtype, device=q.device)
+    if state_out is None:
+        state_out = torch.empty(N, Hv, dv, dk, dtype=torch.float32, device=q.device)
+    need = prefill_workspace_bytes(N, Hv, dk, dv, q.dtype)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().gdn_prefill(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), g.data_ptr(), beta.data_ptr(),
+        state_in.data_ptr() if state_in is not None else None, cu_seqlens.data_ptr(),
+        N, T, Hqk, Hv, dk, dv, float(scale or 0.0), int(chunk), _dtype_code(q),
+        o.data_ptr(), state_out.data_ptr(), ws_ptr, ws_bytes, _stream_handle(stream)))
+    return o, state_out
+
+
+def decode(q, k, v, g, beta, state, *, scale=None, o=None, stream=None):
+    """One decode step: q, k [B, Hqk, dk]; v [B, Hv, dv]; g, beta [B, Hv];
+    state [B, Hv, dv, dk] fp32 updated in place. Returns o [B, Hv, dv]."""
+    _dev(q, "q"); _dev(k, "k", q.dtype); _dev(v, "v", q.dtype)
+    _dev(g, "g", torch.float32); _dev(beta, "beta", torch.float32)
+    _dev(state, "state", torch.float32)
+    B, Hqk, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[2]
+    if o is None:
+        o = torch.empty(B, Hv, dv, dtype=q.dtype, device=q.device)
+    _check(lib().gdn_decode(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), g.data_ptr(), beta.data_ptr(), state.data_ptr(),
+        B, Hqk, Hv, dk, dv, float(scale or 0.0), _dtype_code(q), o.data_ptr(),
+        _stream_handle(stream)))
+    return o
+
+
+def device_error(stream=None) -> None:
+    """Synchronise and raise GdnError if a bounded device wait ran out."""
+    _check(lib().gdn_device_error(_stream_handle(stream)))

@@ -1,0 +1,196 @@
+// C ABI of libgdn.so: argument checks, kernel selection and launches.
+// Declared and documented in include/gdn.h.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "gdn.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "prefill_simt.cuh"
+
+namespace {
+
+thread_local std::string t_last_error;
+
+gdn_status fail(gdn_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+gdn_status fail(gdn_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return s;
+}
+
+gdn_status ok() {
+  t_last_error.clear();
+  return GDN_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+bool head_dim_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+
+gdn_status launch_status(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "%s: launch failed: %s", what, cudaGetErrorString(e));
+  return ok();
+}
+
+// ---------------------------------------------------------------- decode ---
+template <typename TIO, int DK>
+gdn_status launch_decode(const void* q, const void* k, const void* v, const float* g,
+                         const float* beta, float* state, int B, int Hqk, int Hv, int dv,
+                         float scale, void* o, cudaStream_t st) {
+  using Sh = gdn::DecodeShape<DK>;
+  dim3 grid((unsigned)(B * Hv), (unsigned)((dv + Sh::kRowsPerCta - 1) / Sh::kRowsPerCta));
+  gdn::decode_step_kernel<TIO, DK><<<grid, Sh::kWarps * 32, 0, st>>>(
+      static_cast<const TIO*>(q), static_cast<const TIO*>(k), static_cast<const TIO*>(v), g, beta,
+      state, Hqk, Hv, dv, scale, static_cast<TIO*>(o));
+  return launch_status("gdn_decode");
+}
+
+template <typename TIO>
+gdn_status dispatch_decode(const void* q, const void* k, const void* v, const float* g,
+                           const float* beta, float* state, int B, int Hqk, int Hv, int dk,
+                           int dv, float scale, void* o, cudaStream_t st) {
+  switch (dk) {
+    case 16: return launch_decode<TIO, 16>(q, k, v, g, beta, state, B, Hqk, Hv, dv, scale, o, st);
+    case 32: return launch_decode<TIO, 32>(q, k, v, g, beta, state, B, Hqk, Hv, dv, scale, o, st);
+    case 64: return launch_decode<TIO, 64>(q, k, v, g, beta, state, B, Hqk, Hv, dv, scale, o, st);
+    default: return launch_decode<TIO, 128>(q, k, v, g, beta, state, B, Hqk, Hv, dv, scale, o, st);
+  }
+}
+
+// --------------------------------------------------------------- prefill ---
+constexpr size_t kSmemLimit = 227 * 1024;
+
+int simt_slice_rows(int dk, int dv, int C) {
+  // widest state slice whose working set fits in shared memory, at most 32 rows
+  for (int dvp = dv < 32 ? dv : 32; dvp >= 8; dvp /= 2) {
+    if (dv % dvp) continue;
+    if ((size_t)gdn::SimtSmem(C, dk, dvp).total * sizeof(float) <= kSmemLimit) return dvp;
+  }
+  return 0;
+}
+
+template <typename TIO>
+gdn_status launch_prefill_simt(const void* q, const void* k, const void* v, const float* g,
+                               const float* beta, const float* state_in, const int32_t* cu,
+                               int n_seqs, int64_t total_T, int Hqk, int Hv, int dk, int dv,
+                               float scale, int C, void* o, float* state_out, cudaStream_t st) {
+  const int dvp = simt_slice_rows(dk, dv, C);
+  if (dvp == 0)
+    return fail(GDN_ERR_UNSUPPORTED, "gdn_prefill: dk=%d dv=%d chunk=%d does not fit the SIMT kernel", dk,
+                dv, C);
+  const size_t smem = (size_t)gdn::SimtSmem(C, dk, dvp).total * sizeof(float);
+  auto kern = gdn::prefill_simt_kernel<TIO>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "gdn_prefill: %s", cudaGetErrorString(e));
+  dim3 grid((unsigned)(dv / dvp), (unsigned)Hv, (unsigned)n_seqs);
+  kern<<<grid, 256, smem, st>>>(static_cast<const TIO*>(q), static_cast<const TIO*>(k),
+                                static_cast<const TIO*>(v), g, beta, state_in, cu, Hqk, Hv, dk, dv,
+                                dvp, C, scale, static_cast<TIO*>(o), state_out, (long long)total_T);
+  return launch_status("gdn_prefill");
+}
+
+}  // namespace
+
+extern "C" {
+
+int gdn_version(void) { return (0 << 16) | 1; }
+
+const char* gdn_last_error(void) { return t_last_error.c_str(); }
+
+size_t gdn_prefill_workspace_bytes(int n_seqs, int Hv, int dk, int dv, gdn_dtype dtype) {
+  (void)n_seqs; (void)Hv; (void)dk; (void)dv; (void)dtype;
+  return 0;
+}
+
+gdn_status gdn_prefill(const void* q, const void* k, const void* v, const float* g,
+                       const float* beta, const float* state_in, const int32_t* cu_seqlens,
+                       int n_seqs, int64_t total_T, int Hqk, int Hv, int dk, int dv, float scale,
+                       int chunk, gdn_dtype dtype, void* o, float* state_out, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  if (n_seqs < 0) return fail(GDN_ERR_INVALID_ARG, "gdn_prefill: n_seqs=%d < 0", n_seqs);
+  if (total_T < 0 || total_T >= (int64_t(1) << 31))
+    return fail(GDN_ERR_INVALID_ARG, "gdn_prefill: total_T=%lld out of range", (long long)total_T);
+  if (Hqk <= 0 || Hv <= 0 || Hv % Hqk != 0)
+    return fail(GDN_ERR_INVALID_ARG, "gdn_prefill: Hv=%d must be a positive multiple of Hqk=%d", Hv, Hqk);
+  if (!head_dim_ok(dk) || !head_dim_ok(dv))
+    return fail(GDN_ERR_UNSUPPORTED, "gdn_prefill: dk=%d, dv=%d (supported: 16, 32, 64, 128)", dk, dv);
+  if (dtype != GDN_BF16 && dtype != GDN_F32)
+    return fail(GDN_ERR_INVALID_ARG, "gdn_prefill: unknown dtype %d", (int)dtype);
+  if (n_seqs == 0) return ok();
+  if (!cu_seqlens || !state_out)
+    return fail(GDN_ERR_INVALID_ARG, "gdn_prefill: cu_seqlens and state_out must not be NULL");
+  if (total_T > 0 && (!q || !k || !v || !g || !beta || !o))
+    return fail(GDN_ERR_INVALID_ARG, "gdn_prefill: q, k, v, g, beta and o must not be NULL");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(state_out) ||
+      !aligned16(state_in))
+    return fail(GDN_ERR_INVALID_ARG, "gdn_prefill: q, k, v, o and the states must be 16-byte aligned");
+  if (!aligned4(g) || !aligned4(beta) || !aligned4(cu_seqlens))
+    return fail(GDN_ERR_INVALID_ARG, "gdn_prefill: g, beta and cu_seqlens must be 4-byte aligned");
+  const size_t need = gdn_prefill_workspace_bytes(n_seqs, Hv, dk, dv, dtype);
+  if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace)))
+    return fail(GDN_ERR_INVALID_ARG, "gdn_prefill: workspace needs %zu bytes (16-byte aligned), got %zu",
+                need, workspace_bytes);
+  if (scale <= 0.f) scale = 1.0f / sqrtf((float)dk);
+  int C = chunk;
+  if (C == 0) C = (dtype == GDN_BF16 && dk == 128 && dv == 128) ? 64 : 16;
+  if (C != 16 && C != 32 && C != 64)
+    return fail(GDN_ERR_UNSUPPORTED, "gdn_prefill: chunk=%d (supported: 16, 32, 64)", C);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == GDN_F32)
+    return launch_prefill_simt<float>(q, k, v, g, beta, state_in, cu_seqlens, n_seqs, total_T, Hqk,
+                                      Hv, dk, dv, scale, C, o, state_out, st);
+  return launch_prefill_simt<__nv_bfloat16>(q, k, v, g, beta, state_in, cu_seqlens, n_seqs, total_T,
+                                            Hqk, Hv, dk, dv, scale, C, o, state_out, st);
+}
+
+gdn_status gdn_decode(const void* q, const void* k, const void* v, const float* g,
+                      const float* beta, float* state, int B, int Hqk, int Hv, int dk, int dv,
+                      float scale, gdn_dtype dtype, void* o, void* stream) {
+  if (B < 0) return fail(GDN_ERR_INVALID_ARG, "gdn_decode: B=%d < 0", B);
+  if (Hqk <= 0 || Hv <= 0 || Hv % Hqk != 0)
+    return fail(GDN_ERR_INVALID_ARG, "gdn_decode: Hv=%d must be a positive multiple of Hqk=%d", Hv, Hqk);
+  if (!head_dim_ok(dk) || !head_dim_ok(dv))
+    return fail(GDN_ERR_UNSUPPORTED, "gdn_decode: dk=%d, dv=%d (supported: 16, 32, 64, 128)", dk, dv);
+  if (dtype != GDN_BF16 && dtype != GDN_F32)
+    return fail(GDN_ERR_INVALID_ARG, "gdn_decode: unknown dtype %d", (int)dtype);
+  if ((int64_t)B * Hv > 0x7fffffff) return fail(GDN_ERR_INVALID_ARG, "gdn_decode: B*Hv too large");
+  if (B == 0) return ok();
+  if (!q || !k || !v || !g || !beta || !state || !o)
+    return fail(GDN_ERR_INVALID_ARG, "gdn_decode: pointers must not be NULL");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(state))
+    return fail(GDN_ERR_INVALID_ARG, "gdn_decode: q, k, v, o and state must be 16-byte aligned");
+  if (!aligned4(g) || !aligned4(beta))
+    return fail(GDN_ERR_INVALID_ARG, "gdn_decode: g and beta must be 4-byte aligned");
+  if (scale <= 0.f) scale = 1.0f / sqrtf((float)dk);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == GDN_F32)
+    return dispatch_decode<float>(q, k, v, g, beta, state, B, Hqk, Hv, dk, dv, scale, o, st);
+  return dispatch_decode<__nv_bfloat16>(q, k, v, g, beta, state, B, Hqk, Hv, dk, dv, scale, o, st);
+}
+
+gdn_status gdn_device_error(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned int word = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(&word, gdn::g_error_word, sizeof word, 0,
+                                            cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "gdn_device_error: %s", cudaGetErrorString(e));
+  if (word) {
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbolAsync(gdn::g_error_word, &zero, sizeof zero, 0, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "gdn_device_error: %s", cudaGetErrorString(e));
+    return fail(GDN_ERR_DEVICE_TIMEOUT, "a bounded device wait ran out (error word 0x%x)", word);
+  }
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,147 @@
+/*
+ * gdn.h -- C ABI of libgdn.so: the Gated DeltaNet token mixer forward pass
+ * (chunked prefill and single-token decode) on NVIDIA B200 (sm_100a).
+ *
+ * The operation. For every sequence n and value head h the mixer carries a
+ * state S (d_v x d_k, fp32) through the gated delta rule
+ *
+ *     q^_t = q_t / sqrt(|q_t|^2 + 1e-6) * scale,   k^_t = k_t / sqrt(|k_t|^2 + 1e-6)
+ *     S_t  = alpha_t S_{t-1} (I - beta_t k^_t k^_t^T) + beta_t v_t k^_t^T,  alpha_t = exp(g_t)
+ *     o_t  = S_t q^_t
+ *
+ * The Herbert pages name this recurrence as the Gated DeltaNet mixer of
+ * Qwen3.5 ("On descend d'un cran", section "Ce que fait le moteur"; "On
+ * descend d'un cran : #001 un compilateur pour moteur de LLM", section "Un
+ * compilateur, pas une bibliothèque de kernels"), run it in two regimes --
+ * the prompt in blocks at prefill, one row per token at decode -- and fuse
+ * the whole decode step into one launch ("One level down: #004 the same
+ * compiler on Apple's chips", section "Decode"). Their numerical contract is
+ * bf16 activations with f32 accumulation and IEEE rounding, no fast-math
+ * ("On descend d'un cran : #002 le même compilateur sur un GPU", section "Le
+ * contrat numérique"; "One level down: #004", section "In short"). The
+ * equation itself is not printed on the pages; the gated delta rule above is
+ * the reading this library implements, and the fp32 state (rather than the
+ * bf16 state the Metal article mentions) is this library's choice.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor arguments are DEVICE pointers (cudaMalloc'd or equivalent),
+ *     row-major with the innermost index last, contiguous, 16-byte aligned.
+ *     The caller owns every buffer; the library never allocates, frees or
+ *     synchronises (except gdn_device_error, which synchronises the stream).
+ *   - dtype GDN_BF16: q, k, v, o are bf16 (o rounded to nearest even from
+ *     fp32). GDN_F32: q, k, v, o are fp32. g, beta and the states are fp32
+ *     in both cases.
+ *   - Grouped heads: Hv must be a multiple of Hqk; value head h reads
+ *     query/key head floor(h / (Hv / Hqk)) (contiguous groups).
+ *   - g is the log-decay ln(alpha) (<= 0 in normal use); beta is used as given.
+ *   - scale <= 0 selects d_k^-1/2.
+ *   - stream is a cudaStream_t (NULL = legacy default stream). Work is
+ *     enqueued asynchronously; outputs are valid once the stream reaches it.
+ *   - Errors: arguments are checked on the host before anything is enqueued;
+ *     a failed check returns a status, enqueues nothing and writes nothing.
+ *     A launch failure returns GDN_ERR_CUDA. gdn_last_error() returns a
+ *     message for the calling thread's last failure.
+ *   - Every device-side wait is bounded; a wait that runs out sets a device
+ *     error word instead of spinning forever. gdn_device_error() reads it.
+ */
+#ifndef GDN_H
+#define GDN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum gdn_status {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1,    /* null pointer, bad size, misaligned pointer, bad cu_seqlens */
+    GDN_ERR_UNSUPPORTED = 2,    /* valid but unsupported shape/dtype combination */
+    GDN_ERR_CUDA = 3,           /* a CUDA call or launch failed */
+    GDN_ERR_DEVICE_TIMEOUT = 4  /* a bounded device-side wait ran out (gdn_device_error) */
+} gdn_status;
+
+typedef enum gdn_dtype {
+    GDN_BF16 = 0,
+    GDN_F32 = 1
+} gdn_dtype;
+
+/* Library version, (major << 16) | minor. */
+int gdn_version(void);
+
+/*
+ * Bytes of device workspace gdn_prefill needs for this problem (a per-call
+ * work list of (sequence, value head, state slice) items ordered longest
+ * sequence first, and its counter). Depends only on the arguments given.
+ */
+size_t gdn_prefill_workspace_bytes(int n_seqs, int Hv, int dk, int dv, gdn_dtype dtype);
+
+/*
+ * Chunked prefill over packed variable-length sequences.
+ *
+ *   q, k       [total_T, Hqk, dk]   dtype
+ *   v          [total_T, Hv, dv]    dtype
+ *   g, beta    [total_T, Hv]        fp32
+ *   state_in   [n_seqs, Hv, dv, dk] fp32, or NULL for a zero initial state
+ *   cu_seqlens [n_seqs + 1]         int32, DEVICE; cu_seqlens[0] = 0,
+ *                                   non-decreasing, cu_seqlens[n_seqs] = total_T
+ *   o          [total_T, Hv, dv]    dtype (output)
+ *   state_out  [n_seqs, Hv, dv, dk] fp32 (output; may alias state_in exactly)
+ *   workspace  device scratch of at least gdn_prefill_workspace_bytes(...)
+ *              bytes (its contents on entry do not matter)
+ *   chunk      tokens per chunk; 0 selects the default (64 for bf16 with
+ *              dk = dv = 128, else 16). The result does not depend on it
+ *              beyond rounding.
+ *
+ * Supported: GDN_BF16 with dk = dv = 128 and chunk 64 (tensor-core kernel);
+ * GDN_F32 (and GDN_BF16 with other sizes) with dk, dv in {16, 32, 64, 128}
+ * and chunk in {16, 32, 64} (fp32 SIMT kernel). total_T < 2^31.
+ * cu_seqlens is read on the device only; a cu_seqlens that breaks the rules
+ * above is not detected on the host -- sequences with negative length are
+ * treated as empty and tokens past total_T are never read.
+ */
+gdn_status gdn_prefill(const void *q, const void *k, const void *v,
+                       const float *g, const float *beta,
+                       const float *state_in, const int32_t *cu_seqlens,
+                       int n_seqs, int64_t total_T, int Hqk, int Hv, int dk, int dv,
+                       float scale, int chunk, gdn_dtype dtype,
+                       void *o, float *state_out,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * One decode step for B independent sequences, one token each; the fused
+ * step of "One level down: #004 the same compiler on Apple's chips",
+ * section "Decode": L2-normalise q and k, decay, rank-1 delta update and
+ * the o = S q readout in one launch that streams each state once.
+ *
+ *   q, k    [B, Hqk, dk]     dtype
+ *   v       [B, Hv, dv]      dtype
+ *   g, beta [B, Hv]          fp32
+ *   state   [B, Hv, dv, dk]  fp32, updated in place
+ *   o       [B, Hv, dv]      dtype (output)
+ *
+ * Supported: dk = 128 (any dtype), dv any multiple of 8 up to 128... in
+ * practice dk in {16, 32, 64, 128} and dv a multiple of 8.
+ */
+gdn_status gdn_decode(const void *q, const void *k, const void *v,
+                      const float *g, const float *beta, float *state,
+                      int B, int Hqk, int Hv, int dk, int dv,
+                      float scale, gdn_dtype dtype, void *o, void *stream);
+
+/* Message describing the calling thread's most recent failure ("" if none). */
+const char *gdn_last_error(void);
+
+/*
+ * Synchronise `stream` and read, then clear, the device error word of the
+ * current device. Returns GDN_ERR_DEVICE_TIMEOUT if a bounded wait ran out
+ * in any kernel since the last call, GDN_ERR_CUDA if synchronisation failed,
+ * else GDN_OK. Meant for tests and debugging; not needed in normal use.
+ */
+gdn_status gdn_device_error(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H */

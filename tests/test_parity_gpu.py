@@ -1,0 +1,178 @@
+"""GPU parity: the CUDA library against the fp64 oracle, element by element.
+
+Every case feeds the same seeded inputs to both sides. Outputs and states
+are pre-filled with NaN so an element the kernel fails to write fails the
+comparison. Two gates are applied:
+
+  * the absolute max-error tolerance of the workload (fp32 tiny: 1e-4;
+    bf16 prefill/decode: o <= 2e-2, state <= 1e-2; long prefill: o <= 3e-2,
+    state <= 2e-2);
+  * the relative gate of the Herbert Metal article's correctness check
+    ("One level down: #004 the same compiler on Apple's chips", section "The
+    night the engine chose wrong"): max error <= 1/64 of the largest |value|
+    of the reference, which is much tighter than the absolute bounds for o.
+
+Full-size workloads are compared on a sample of value heads (all tokens of
+those heads), which the oracle computes exactly like the full problem.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+gdn = pytest.importorskip("gated_deltanet_linear_21_b200")
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _max_err(gpu, ref, sel=None):
+    a = gpu.detach().to("cpu", torch.float64).numpy()
+    if sel is not None:
+        a, ref = a[sel], ref[sel]
+    assert not np.isnan(a).any(), "kernel left unwritten (NaN) elements"
+    return float(np.abs(a - ref).max()) if a.size else 0.0, float(np.abs(ref).max()) if a.size else 0.0
+
+
+def _gate(name, err, ref_max, tol, rel=1 / 64):
+    assert err <= tol, f"{name}: max abs error {err:.3e} > {tol:.1e}"
+    assert err <= rel * ref_max + 1e-7, f"{name}: max abs error {err:.3e} > 1/64 of max |ref| {ref_max:.3e}"
+
+
+def run_prefill(x, chunk=0, heads=None, state_in_device=True, alias=False):
+    d = {kk: (vv.to(DEV) if isinstance(vv, torch.Tensor) else vv) for kk, vv in x.items()}
+    T, Hv, dv = d["v"].shape
+    N = d["cu_seqlens"].numel() - 1
+    dk = d["q"].shape[2]
+    o = torch.full((T, Hv, dv), float("nan"), dtype=d["q"].dtype, device=DEV)
+    if alias:
+        s_in = d["state_in"].clone() if d["state_in"] is not None else torch.zeros(N, Hv, dv, dk, device=DEV)
+        s_out = s_in
+    else:
+        s_in = d["state_in"]
+        s_out = torch.full((N, Hv, dv, dk), float("nan"), dtype=torch.float32, device=DEV)
+    gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], s_in, d["cu_seqlens"], chunk=chunk,
+                o=o, state_out=s_out)
+    torch.cuda.synchronize()
+    gdn.device_error()
+    ro, rs = oracle.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], x["state_in"], x["cu_seqlens"],
+                            heads=heads)
+    return o, s_out, ro, rs
+
+
+def check_prefill(x, tol_o, tol_s, chunk=0, heads=None, alias=False):
+    o, s, ro, rs = run_prefill(x, chunk=chunk, heads=heads, alias=alias)
+    sel_o = (slice(None), slice(heads[0], heads[1])) if heads else None
+    sel_s = (slice(None), slice(heads[0], heads[1])) if heads else None
+    eo, mo = _max_err(o, ro, sel_o)
+    es, ms = _max_err(s, rs, sel_s)
+    print(f"o err {eo:.3e} (max|o| {mo:.3e})  state err {es:.3e} (max|S| {ms:.3e})")
+    _gate("o", eo, mo, tol_o)
+    _gate("state", es, ms, tol_s)
+    return eo, es
+
+
+# ------------------------------------------------------------------ decode ---
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("dk,dv", [(16, 16), (32, 64), (64, 128), (128, 128), (128, 32)])
+def test_decode_small(dtype, dk, dv):
+    B, Hqk, Hv = 3, 2, 4
+    state = workloads.decode_state(B, Hv, dk, std=0.05, dv=dv)
+    ref_state = state.double().numpy().copy()
+    sd = state.to(DEV)
+    tol = 2e-2 if dtype == torch.bfloat16 else 1e-5
+    for step in range(5):
+        x = workloads.decode_step_inputs(step, B, Hqk, Hv, dk, dtype, dv=dv)
+        o = torch.full((B, Hv, dv), float("nan"), dtype=dtype, device=DEV)
+        gdn.decode(x["q"].to(DEV), x["k"].to(DEV), x["v"].to(DEV), x["g"].to(DEV), x["beta"].to(DEV),
+                   sd, o=o)
+        ro, ref_state = oracle.decode(x["q"], x["k"], x["v"], x["g"], x["beta"], ref_state)
+        eo, mo = _max_err(o, ro)
+        _gate("o", eo, mo, tol)
+    es, ms = _max_err(sd, ref_state)
+    _gate("state", es, ms, 1e-2 if dtype == torch.bfloat16 else 1e-5)
+
+
+def test_decode_workload_1000_steps_sampled_heads():
+    """64 sequences x 32 value heads, d=128, 1000 consecutive steps; o checked at
+    every step and the state after the last one, on value heads 0..3."""
+    w = workloads.workload("decode")
+    heads = (0, 4)
+    state = workloads.decode_state(w.batch, w.Hv, w.d, std=w.state_std)
+    ref = state.double().numpy().copy()
+    sd = state.to(DEV)
+    worst_o = 0.0
+    for step in range(w.steps):
+        x = workloads.decode_step_inputs(step, w.batch, w.Hqk, w.Hv, w.d)
+        o = gdn.decode(x["q"].to(DEV), x["k"].to(DEV), x["v"].to(DEV), x["g"].to(DEV), x["beta"].to(DEV), sd)
+        ro, ref = oracle.decode(x["q"], x["k"], x["v"], x["g"], x["beta"], ref, heads=heads)
+        eo, mo = _max_err(o, ro, (slice(None), slice(*heads)))
+        worst_o = max(worst_o, eo)
+        assert eo <= w.tol_o, f"step {step}: o err {eo:.3e}"
+    es, ms = _max_err(sd, ref, (slice(None), slice(*heads)))
+    print(f"decode 1000 steps: worst o err {worst_o:.3e}, state err {es:.3e} (max|S| {ms:.3e})")
+    assert es <= w.tol_state
+    assert not torch.isnan(sd).any()
+
+
+# ----------------------------------------------------------------- prefill ---
+
+def test_prefill_tiny_fp32_workload():
+    w = workloads.workload("tiny")
+    check_prefill(workloads.inputs_for(w), w.tol_o, w.tol_state, chunk=w.chunk)
+
+
+@pytest.mark.parametrize("lengths", [[1], [63], [64], [65], [197], [5, 130, 1, 64, 77], [0, 40, 0]])
+def test_prefill_small_bf16_ragged(lengths):
+    x = workloads.prefill_inputs(lengths, Hqk=2, Hv=4, d=128, seed=77 + sum(lengths), state_std=0.05)
+    check_prefill(x, 2e-2, 1e-2)
+
+
+@pytest.mark.parametrize("d", [16, 32, 64])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_prefill_small_heads_simt(d, dtype):
+    x = workloads.prefill_inputs([50, 17], Hqk=1, Hv=2, d=d, dtype=dtype, seed=91 + d, state_std=0.05)
+    tol = 2e-2 if dtype == torch.bfloat16 else 1e-4
+    for chunk in (16, 32, 64):
+        check_prefill(x, tol, tol if dtype == torch.float32 else 1e-2, chunk=chunk)
+
+
+def test_prefill_state_in_aliases_state_out():
+    x = workloads.prefill_inputs([100, 29], Hqk=2, Hv=4, d=128, seed=5, state_std=0.05)
+    check_prefill(x, 2e-2, 1e-2, alias=True)
+
+
+def test_prefill_continuation_and_decode_agree_with_one_run():
+    x = workloads.prefill_inputs([150], Hqk=2, Hv=4, d=128, seed=6, state_std=0.05)
+    d = {kk: (vv.to(DEV) if isinstance(vv, torch.Tensor) else vv) for kk, vv in x.items()}
+    o_all, s_all = gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["state_in"], d["cu_seqlens"])
+    sl = lambda t, a, b: t[a:b].contiguous()
+    o1, s1 = gdn.prefill(*(sl(d[n], 0, 100) for n in ("q", "k", "v", "g", "beta")), d["state_in"])
+    o2, s2 = gdn.prefill(*(sl(d[n], 100, 140) for n in ("q", "k", "v", "g", "beta")), s1)
+    s3 = s2.clone()
+    outs = []
+    for t in range(140, 150):
+        outs.append(gdn.decode(*(sl(d[n], t, t + 1) for n in ("q", "k", "v", "g", "beta")), s3))
+    o_cat = torch.cat([o1, o2] + outs)
+    assert (o_cat.float() - o_all.float()).abs().max().item() <= 2e-2
+    assert (s3 - s_all).abs().max().item() <= 1e-2
+
+
+def test_prefill_workload_qwen08b_layer_full():
+    """1 x 4096 tokens, 16 q/k and 16 v heads, d=128, bf16: every element."""
+    w = workloads.workload("prefill")
+    check_prefill(workloads.inputs_for(w), w.tol_o, w.tol_state)
+
+
+@pytest.mark.parametrize("T", [32768, 81920])
+def test_prefill_workload_long_sampled_heads(T):
+    w = workloads.workload("long", T=T)
+    check_prefill(workloads.inputs_for(w), w.tol_o, w.tol_state, heads=(0, 2) if T > 40000 else (0, 3))
+
+
+def test_prefill_workload_varlen_sampled_heads():
+    w = workloads.workload("varlen")
+    check_prefill(workloads.inputs_for(w), w.tol_o, w.tol_state, heads=(0, 4))
