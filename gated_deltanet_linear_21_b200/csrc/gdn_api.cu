@@ -9,6 +9,10 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "prefill_simt.cuh"
+#include "prefill_tc.cuh"
+
+#include <cudaTypedefs.h>
+#include <cstdlib>
 
 namespace {
 
@@ -97,6 +101,78 @@ gdn_status launch_prefill_simt(const void* q, const void* k, const void* v, cons
   return launch_status("gdn_prefill");
 }
 
+// ------------------------------------------------- tensor-core prefill ---
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 3-D bf16 map over a token-major [T][H][D] tensor: dims (D, H, T), box (box_d, 1, 64).
+bool make_map(CUtensorMap* m, const void* base, int D, int H, int T, int box_d) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+  cuuint32_t box[3] = {(cuuint32_t)box_d, 1, (cuuint32_t)gdn::tc::kC};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const int row_bytes = box_d * 2;
+  CUtensorMapSwizzle sw = row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                          : row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                            : CU_TENSOR_MAP_SWIZZLE_32B;
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Rows of the state per CTA: enough CTAs to cover the 148 SMs once.
+int tc_slice_rows(int n_seqs, int Hv) {
+  if (const char* env = getenv("GDN_TC_SLICE")) {
+    const int v = atoi(env);
+    if (v == 16 || v == 32 || v == 64) return v;
+  }
+  const long chains = (long)n_seqs * Hv;
+  if (chains <= 18) return 16;
+  if (chains <= 37) return 32;
+  return 64;
+}
+
+template <int DVP>
+gdn_status launch_tc(const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm, const float* g,
+                     const float* beta, const float* state_in, const int32_t* cu, int n_seqs, int Hqk,
+                     int Hv, float scale, void* o, float* state_out, int total_T, cudaStream_t st) {
+  const size_t smem = gdn::tc::Smem<DVP>::kAlloc;
+  auto kern = gdn::tc::prefill_tc_kernel<DVP>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "gdn_prefill: %s", cudaGetErrorString(e));
+  dim3 grid(gdn::tc::kD / DVP, (unsigned)Hv, (unsigned)n_seqs);
+  kern<<<grid, gdn::tc::kThreads, smem, st>>>(qm, km, vm, g, beta, state_in, cu, Hqk, Hv, scale,
+                                              static_cast<__nv_bfloat16*>(o), state_out, total_T);
+  return launch_status("gdn_prefill");
+}
+
+gdn_status launch_prefill_tc(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                             const float* state_in, const int32_t* cu, int n_seqs, int64_t total_T, int Hqk,
+                             int Hv, float scale, void* o, float* state_out, cudaStream_t st) {
+  const int dvp = tc_slice_rows(n_seqs, Hv);
+  CUtensorMap qm, km, vm;
+  if (!make_map(&qm, q, 128, Hqk, (int)total_T, 64) || !make_map(&km, k, 128, Hqk, (int)total_T, 64) ||
+      !make_map(&vm, v, 128, Hv, (int)total_T, dvp))
+    return fail(GDN_ERR_CUDA, "gdn_prefill: cuTensorMapEncodeTiled unavailable or failed");
+  switch (dvp) {
+    case 16: return launch_tc<16>(qm, km, vm, g, beta, state_in, cu, n_seqs, Hqk, Hv, scale, o, state_out, (int)total_T, st);
+    case 32: return launch_tc<32>(qm, km, vm, g, beta, state_in, cu, n_seqs, Hqk, Hv, scale, o, state_out, (int)total_T, st);
+    default: return launch_tc<64>(qm, km, vm, g, beta, state_in, cu, n_seqs, Hqk, Hv, scale, o, state_out, (int)total_T, st);
+  }
+}
+
 }  // namespace
 
 extern "C" {
@@ -144,6 +220,9 @@ gdn_status gdn_prefill(const void* q, const void* k, const void* v, const float*
   if (C != 16 && C != 32 && C != 64)
     return fail(GDN_ERR_UNSUPPORTED, "gdn_prefill: chunk=%d (supported: 16, 32, 64)", C);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == GDN_BF16 && dk == 128 && dv == 128 && C == 64 && total_T > 0)
+    return launch_prefill_tc(q, k, v, g, beta, state_in, cu_seqlens, n_seqs, total_T, Hqk, Hv, scale, o,
+                             state_out, st);
   if (dtype == GDN_F32)
     return launch_prefill_simt<float>(q, k, v, g, beta, state_in, cu_seqlens, n_seqs, total_T, Hqk,
                                       Hv, dk, dv, scale, C, o, state_out, st);
