@@ -1,0 +1,502 @@
+"""Benchmark of the Gated DeltaNet mixer forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload prefill|long|varlen|decode] [--no-extras]
+
+One step is one gdn_prefill call over the workload: the whole chunked-prefill
+path (q/k normalisation, decay cumsum, UT transform, intra-chunk attention,
+inter-chunk state passing) for a Qwen3.5-0.8B-like mixer layer, 1 x 4096
+tokens, 16 q/k and 16 v heads, d = 128, bf16, chunk 64. The JSON line also
+carries the 1000-step decode workload (64 sequences x 32 v heads) and the
+32768-token long prefill as sub-objects, each with its own roofline.
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own copy of
+the workload (independent sequences, no data exchange), so scaling is weak
+and the value is the sum over ranks divided by the slowest rank's time.
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded
+sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+import workloads  # noqa: E402
+
+METRIC = "prefill tokens/s & decode steps/s per mixer layer; % tensor/HBM roofline"
+DATA = ("synthetic: seeded q, k, v ~ N(0,1) (bf16), alpha = sigmoid(N(3,1)) passed as "
+        "g = log(alpha), beta = sigmoid(N(0,1)), fp32 gates")
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------- helpers ---
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def prefill_flops_per_token_head(C=64, d=128):
+    """Algorithmic flops of the chunked method per token per value head,
+    triangle-aware: KK^T and QK^T strictly/inclusive lower (C^2 d each per
+    chunk), T [beta V | beta gamma K] (2 C^2 d), (M o QK^T) U (C^2 d) and the
+    three d x d x C state products (6 C d^2), i.e. 5 C d + 6 d^2 per token."""
+    return 5 * C * d + 6 * d * d
+
+
+def prefill_bytes(T, Hqk, Hv, d, N, state_in):
+    """Algorithmic HBM bytes of one prefill: every input read once, every output written once."""
+    b = T * Hqk * d * 2 * 2 + T * Hv * d * 2 + T * Hv * d * 2 + T * Hv * 4 * 2
+    b += N * Hv * d * d * 4 * (2 if state_in else 1) + (N + 1) * 4
+    return b
+
+
+def decode_bytes(B, Hqk, Hv, d):
+    """Algorithmic HBM bytes of one decode step: state read + written, q, k, v, o, gates."""
+    return B * Hv * d * d * 4 * 2 + B * Hqk * d * 2 * 2 + B * Hv * d * 2 * 2 + B * Hv * 4 * 2
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gated_deltanet_linear_21_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_record(kernel):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(kernel)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("source_hash") != kernel_source_hash():
+        return None
+    return rec
+
+
+class ClockSampler:
+    """Samples the SM clock and the clock-event (throttle) reasons through NVML
+    every ~2 ms while a timed region runs (reading only; nothing is changed)."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
+
+    def __init__(self, device_index):
+        self.device_index = device_index
+        self.samples = []
+        self.max_mhz = None
+        self._stop = None
+
+    def _handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.device_index)
+        try:
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.device_index)
+
+    def __enter__(self):
+        import threading
+        try:
+            self.nvml, self.handle = self._handle()
+            self.max_mhz = self.nvml.nvmlDeviceGetMaxClockInfo(self.handle, self.nvml.NVML_CLOCK_SM)
+        except Exception:
+            self.handle = None
+            return self
+        self._stop = threading.Event()
+
+        def loop():
+            while not self._stop.is_set():
+                try:
+                    mhz = self.nvml.nvmlDeviceGetClockInfo(self.handle, self.nvml.NVML_CLOCK_SM)
+                    rs = self.nvml.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                    self.samples.append((mhz, rs))
+                except Exception:
+                    pass
+                self._stop.wait(0.002)
+
+        self._thread = threading.Thread(target=loop, daemon=True)
+        self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._stop is not None:
+            self._stop.set()
+            self._thread.join(timeout=2)
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"]}
+        reasons = set()
+        for _, rs in self.samples:
+            for name, const in self.REASONS:
+                if rs & getattr(self.nvml, const, 0):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(self.samples)}
+
+
+def timed(fn, stream):
+    """Device time (ms) of fn() on `stream`, bracketed by synchronisation."""
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b)
+
+
+# ------------------------------------------------------------ our workload ---
+def device_prefill_inputs(lengths, Hqk, Hv, d, seed, device, state_std=0.0):
+    """Seeded inputs generated on the device (same distributions as workloads.py)."""
+    gen = torch.Generator(device=device).manual_seed(seed)
+    T = sum(lengths)
+    q = torch.randn(T, Hqk, d, generator=gen, device=device).to(torch.bfloat16)
+    k = torch.randn(T, Hqk, d, generator=gen, device=device).to(torch.bfloat16)
+    v = torch.randn(T, Hv, d, generator=gen, device=device).to(torch.bfloat16)
+    x = torch.randn(T, Hv, generator=gen, device=device, dtype=torch.float64) + 3.0
+    y = torch.randn(T, Hv, generator=gen, device=device, dtype=torch.float64)
+    g = torch.nn.functional.logsigmoid(x).float()
+    beta = torch.sigmoid(y).float()
+    cu = torch.zeros(len(lengths) + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(torch.tensor(lengths), 0)
+    s0 = None
+    if state_std > 0:
+        s0 = torch.randn(len(lengths), Hv, d, d, generator=gen, device=device) * state_std
+    return dict(q=q, k=k, v=v, g=g, beta=beta, cu_seqlens=cu.to(device), state_in=s0)
+
+
+def run_prefill_bench(gdn, w, steps, warmup, device, rank, sampler=None):
+    stream = torch.cuda.current_stream()
+    T = w.total_tokens
+    one = prefill_bytes(T, w.Hqk, w.Hv, w.d, len(w.lengths), w.state_std > 0)
+    copies = max(2, -(-3 * L2_BYTES // one))   # rotate inputs over > 3x L2
+    bufs = [device_prefill_inputs(w.lengths, w.Hqk, w.Hv, w.d, 7919 * rank + 31 * i + w.index,
+                                  device, w.state_std) for i in range(copies)]
+    outs = [(torch.empty(T, w.Hv, w.d, dtype=torch.bfloat16, device=device),
+             torch.empty(len(w.lengths), w.Hv, w.d, w.d, device=device)) for _ in range(copies)]
+
+    def step(i):
+        x = bufs[i % copies]
+        o, s = outs[i % copies]
+        gdn.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], x["state_in"], x["cu_seqlens"],
+                    o=o, state_out=s)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    # capture the K steps once, replay on the device without host gaps
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for i in range(steps):
+            step(i)
+    torch.cuda.synchronize()
+    graph.replay()   # untimed replay: first-replay costs
+    torch.cuda.synchronize()
+    if sampler is not None:
+        with sampler:
+            ms = timed(graph.replay, stream) / steps
+    else:
+        ms = timed(graph.replay, stream) / steps
+    return dict(ms=ms, tokens=T, bytes=one, copies=copies, graph=graph)
+
+
+def run_decode_bench(gdn, w, steps_timed, warmup, device, rank, sampler=None):
+    stream = torch.cuda.current_stream()
+    B, Hqk, Hv, d = w.batch, w.Hqk, w.Hv, w.d
+    gen = torch.Generator(device=device).manual_seed(workloads.SEED_DECODE_STEP + 7919 * rank)
+    n = steps_timed
+    qs = torch.randn(n, B, Hqk, d, generator=gen, device=device).to(torch.bfloat16)
+    ks = torch.randn(n, B, Hqk, d, generator=gen, device=device).to(torch.bfloat16)
+    vs = torch.randn(n, B, Hv, d, generator=gen, device=device).to(torch.bfloat16)
+    gs = torch.nn.functional.logsigmoid(torch.randn(n, B, Hv, generator=gen, device=device) + 3.0)
+    bs = torch.sigmoid(torch.randn(n, B, Hv, generator=gen, device=device))
+    state = torch.randn(B, Hv, d, d, generator=gen, device=device) * w.state_std
+    o = torch.empty(B, Hv, d, dtype=torch.bfloat16, device=device)
+
+    def run(a, b):
+        for t in range(a, b):
+            gdn.decode(qs[t], ks[t], vs[t], gs[t], bs[t], state, o=o)
+
+    run(0, min(warmup, n))
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        run(0, n)
+    graph.replay()
+    torch.cuda.synchronize()
+    if sampler is not None:
+        with sampler:
+            ms = timed(graph.replay, stream) / n
+    else:
+        ms = timed(graph.replay, stream) / n
+    return dict(ms=ms, bytes=decode_bytes(B, Hqk, Hv, d), steps=n)
+
+
+def run_e2e(gdn, w, steps, device):
+    """Same prefill through the public API with inputs in pinned host memory:
+    H2D of q, k, v, g, beta, the call, and D2H of o and the final states."""
+    stream = torch.cuda.current_stream()
+    x = workloads.inputs_for(w) if w.total_tokens <= 8192 else None
+    if x is None:
+        x = {kk: (vv.cpu() if isinstance(vv, torch.Tensor) else vv)
+             for kk, vv in device_prefill_inputs(w.lengths, w.Hqk, w.Hv, w.d, 11, device).items()}
+    host = {kk: vv.pin_memory() for kk, vv in x.items() if isinstance(vv, torch.Tensor)}
+    dev = {kk: torch.empty_like(vv, device=device) for kk, vv in host.items()}
+    T, N = w.total_tokens, len(w.lengths)
+    o_h = torch.empty(T, w.Hv, w.d, dtype=torch.bfloat16).pin_memory()
+    s_h = torch.empty(N, w.Hv, w.d, w.d).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = o_h.numel() * o_h.element_size() + s_h.numel() * s_h.element_size()
+
+    def step():
+        for kk in host:
+            dev[kk].copy_(host[kk], non_blocking=True)
+        o, s = gdn.prefill(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], dev.get("state_in"),
+                           dev["cu_seqlens"])
+        o_h.copy_(o, non_blocking=True)
+        s_h.copy_(s, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    ms = timed(lambda: [step() for _ in range(steps)], stream) / steps
+    return dict(ms=ms, h2d=h2d, d2h=d2h, tokens=T)
+
+
+def cpu_baseline(w, budget_s=10.0):
+    """The fp64 oracle as it stands, on the host cores, over whole copies of the
+    workload until about budget_s seconds have passed."""
+    import oracle
+    x = workloads.inputs_for(w)
+    cores = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], x["state_in"], x["cu_seqlens"],
+                       n_threads=cores)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or reps >= 50:
+            break
+    return dict(value=reps * w.total_tokens / el, unit="tokens/s", cores=cores, kind="oracle",
+                sample=f"{reps} full pass(es) of the workload ({w.total_tokens} tokens x {w.Hv} heads), "
+                       f"{el:.1f} s wall")
+
+
+def workload_config(w, copies=None, n=1):
+    if w.kind == "decode":
+        return {"workload": f"{w.name}: {w.batch} sequences x 1 token, {w.steps} consecutive steps, "
+                            f"Hqk={w.Hqk} Hv={w.Hv} d_k=d_v={w.d} {w.dtype}, fp32 state in place",
+                "global_batch": w.batch * n, "seq_len": 1,
+                "parallelism": f"dp{n} (independent sequences per rank, no exchange)"}
+    cfg = {"workload": f"{w.name}: {w.kind} "
+                       + (f"T={w.lengths[0]}" if len(w.lengths) == 1 else f"{len(w.lengths)} seqs "
+                          f"(total {w.total_tokens} tokens)")
+                       + f" Hqk={w.Hqk} Hv={w.Hv} d_k=d_v={w.d} {w.dtype} chunk={w.chunk}",
+           "global_batch": len(w.lengths) * n, "seq_len": w.total_tokens,
+           "parallelism": f"dp{n} (independent sequences per rank, no exchange)"}
+    if copies:
+        cfg["l2"] = f"inputs rotated over {copies} copies (> 3x the 126 MB L2)"
+    return cfg
+
+
+def roofline_tensor(flops, ms, pk, kind, key="bf16_tflops", traffic=None):
+    achieved = flops / (ms * 1e-3) / 1e12
+    peak = pk[key]
+    return {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4), "traffic": traffic, "peak_kind": f"{key} ({kind})"}
+
+
+def roofline_hbm(nbytes, ms, pk, kind, traffic=None):
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    peak = pk["hbm_gbs"]
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": traffic, "peak_kind": f"hbm_gbs ({kind})"}
+
+
+# -------------------------------------------------------------------- main ---
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="prefill", choices=["prefill", "long", "varlen", "decode"])
+    ap.add_argument("--no-extras", action="store_true", help="main workload only (for profiling)")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = workloads.workload(args.workload)
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        times = []
+        cores = os.cpu_count() or 1
+        import oracle
+        x = workloads.inputs_for(w) if w.kind == "prefill" else None
+        if w.kind == "decode":
+            state = workloads.decode_state(w.batch, w.Hv, w.d).double().numpy()
+            xs = [workloads.decode_step_inputs(s, w.batch, w.Hqk, w.Hv, w.d) for s in range(4)]
+
+        def ref_step(i):
+            if w.kind == "prefill":
+                oracle.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], x["state_in"], x["cu_seqlens"],
+                               n_threads=cores)
+            else:
+                xi = xs[i % 4]
+                oracle.decode(xi["q"], xi["k"], xi["v"], xi["g"], xi["beta"], state, n_threads=cores)
+
+        for i in range(args.warmup):
+            ref_step(i)
+        t0 = time.perf_counter()
+        for i in range(args.steps):
+            ref_step(i)
+        el = time.perf_counter() - t0
+        ms = el * 1e3 / args.steps
+        if w.kind == "prefill":
+            value, unit = w.total_tokens / (ms * 1e-3), "tokens/s"
+        else:
+            value, unit = 1.0 / (ms * 1e-3), "steps/s"
+        sample = (f"{args.steps} step(s) of the whole workload, fp64 C oracle, OpenMP over "
+                  f"(sequence, head), {cores} threads")
+        line = {"impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": DATA,
+                "config": workload_config(w),
+                "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
+                                 "sample": sample},
+                "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    # ------------------------------------------------------------ our arm ---
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", device_id=device, timeout=datetime.timedelta(seconds=120))
+    import gated_deltanet_linear_21_b200 as gdn
+
+    pk, pk_kind = peaks()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        import torch.distributed as dist
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier(device_ids=[local])
+        torch.cuda.synchronize()
+
+    if w.kind == "prefill":
+        clk = ClockSampler(local)
+        barrier()
+        r = run_prefill_bench(gdn, w, args.steps, args.warmup, device, rank, clk)
+        barrier()
+        ms = max_over_ranks(r["ms"])
+        value = world * r["tokens"] / (ms * 1e-3)
+        flops = prefill_flops_per_token_head(w.chunk, w.d) * r["tokens"] * w.Hv
+        tr = traffic_record("prefill_tc")
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": DATA,
+                "config": workload_config(w, r["copies"], world),
+                "roofline": roofline_tensor(flops, r["ms"], pk, pk_kind,
+                                            traffic=tr["bytes_per_launch"] if tr else None),
+                "roofline_hbm_view": roofline_hbm(r["bytes"], r["ms"], pk, pk_kind),
+                "gpu_launches": args.steps, "clocks": clk.summary()}
+        del r["graph"]
+    else:
+        clk = ClockSampler(local)
+        barrier()
+        r = run_decode_bench(gdn, w, w.steps, args.warmup, device, rank, clk)
+        barrier()
+        ms = max_over_ranks(r["ms"])
+        tr = traffic_record("decode")
+        line = {"metric": METRIC, "value": world / (ms * 1e-3), "unit": "steps/s", "n_gpus": world,
+                "steps": r["steps"], "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": DATA,
+                "config": dict(workload_config(w, None, world),
+                               l2="state 134 MB > 126 MB L2; fresh q/k/v buffers every step"),
+                "roofline": roofline_hbm(r["bytes"], r["ms"], pk, pk_kind,
+                                         traffic=tr["bytes_per_launch"] if tr else None),
+                "gpu_launches": r["steps"], "clocks": clk.summary()}
+
+    if not args.no_extras and w.kind == "prefill":
+        # decode workload: 1000 consecutive steps, fresh tokens each step
+        wd = workloads.workload("decode")
+        rd = run_decode_bench(gdn, wd, wd.steps, args.warmup, device, rank)
+        msd = max_over_ranks(rd["ms"])
+        trd = traffic_record("decode")
+        line["decode"] = {"value": world / (msd * 1e-3), "unit": "steps/s", "ms_per_step": msd,
+                          "steps": rd["steps"], "gpu_launches": rd["steps"],
+                          "config": workload_config(wd, None, world),
+                          "roofline": roofline_hbm(rd["bytes"], rd["ms"], pk, pk_kind,
+                                                   traffic=trd["bytes_per_launch"] if trd else None)}
+        # long prompt: 32768 tokens, 16 q/k and 32 v heads
+        wl = workloads.workload("long")
+        nl = max(2, args.steps // 4)
+        rl = run_prefill_bench(gdn, wl, nl, args.warmup, device, rank)
+        del rl["graph"]
+        msl = max_over_ranks(rl["ms"])
+        fl = prefill_flops_per_token_head(wl.chunk, wl.d) * rl["tokens"] * wl.Hv
+        line["long_prefill"] = {"value": world * rl["tokens"] / (msl * 1e-3), "unit": "tokens/s",
+                                "ms_per_step": msl, "steps": nl, "gpu_launches": nl,
+                                "config": workload_config(wl, rl["copies"], world),
+                                "roofline": roofline_tensor(fl, rl["ms"], pk, pk_kind),
+                                "roofline_hbm_view": roofline_hbm(rl["bytes"], rl["ms"], pk, pk_kind)}
+
+    if w.kind == "prefill":
+        e = run_e2e(gdn, w, max(3, args.steps // 2), device)
+        ems = max_over_ranks(e["ms"])
+        line["e2e"] = {"value": world * e["tokens"] / (ems * 1e-3), "unit": "tokens/s",
+                       "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"]}
+    if rank == 0 and world == 1 and not args.no_extras and w.kind == "prefill":
+        line["cpu_baseline"] = cpu_baseline(w)
+
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

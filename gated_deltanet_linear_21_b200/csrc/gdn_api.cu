@@ -3,7 +3,10 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
+#include <set>
 #include <string>
+#include <utility>
 
 #include "gdn.h"
 #include "common.cuh"
@@ -38,6 +41,25 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 bool head_dim_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
 
+// Allow a kernel the full opt-in shared memory, once per (kernel, device), so
+// that later calls (including ones inside CUDA-graph capture) only launch.
+constexpr size_t kSmemOptIn = 227 * 1024;
+template <typename F>
+gdn_status allow_smem(F* kern, const char* what) {
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_pair(reinterpret_cast<const void*>(kern), dev);
+  if (done.count(key)) return GDN_OK;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemOptIn);
+  if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  done.insert(key);
+  return GDN_OK;
+}
+
 gdn_status launch_status(const char* what) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "%s: launch failed: %s", what, cudaGetErrorString(e));
@@ -70,7 +92,7 @@ gdn_status dispatch_decode(const void* q, const void* k, const void* v, const fl
 }
 
 // --------------------------------------------------------------- prefill ---
-constexpr size_t kSmemLimit = 227 * 1024;
+constexpr size_t kSmemLimit = kSmemOptIn;
 
 int simt_slice_rows(int dk, int dv, int C) {
   // widest state slice whose working set fits in shared memory, at most 32 rows
@@ -92,8 +114,7 @@ gdn_status launch_prefill_simt(const void* q, const void* k, const void* v, cons
                 dv, C);
   const size_t smem = (size_t)gdn::SimtSmem(C, dk, dvp).total * sizeof(float);
   auto kern = gdn::prefill_simt_kernel<TIO>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "gdn_prefill: %s", cudaGetErrorString(e));
+  if (gdn_status s = allow_smem(kern, "gdn_prefill")) return s;
   dim3 grid((unsigned)(dv / dvp), (unsigned)Hv, (unsigned)n_seqs);
   kern<<<grid, 256, smem, st>>>(static_cast<const TIO*>(q), static_cast<const TIO*>(k),
                                 static_cast<const TIO*>(v), g, beta, state_in, cu, Hqk, Hv, dk, dv,
@@ -150,8 +171,7 @@ gdn_status launch_tc(const CUtensorMap& qm, const CUtensorMap& km, const CUtenso
                      int Hv, float scale, void* o, float* state_out, int total_T, cudaStream_t st) {
   const size_t smem = gdn::tc::Smem<DVP>::kAlloc;
   auto kern = gdn::tc::prefill_tc_kernel<DVP>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "gdn_prefill: %s", cudaGetErrorString(e));
+  if (gdn_status s = allow_smem(kern, "gdn_prefill")) return s;
   dim3 grid(gdn::tc::kD / DVP, (unsigned)Hv, (unsigned)n_seqs);
   kern<<<grid, gdn::tc::kThreads, smem, st>>>(qm, km, vm, g, beta, state_in, cu, Hqk, Hv, scale,
                                               static_cast<__nv_bfloat16*>(o), state_out, total_T);

@@ -31,10 +31,17 @@
 // rewritten; the L2 norms come from the diagonal of [k;q][k;q]^T and are
 // folded into scalings of the small 64 x 64 matrices.
 //
-// One CTA of 128 threads owns one (sequence, value head, slice of DVP state
-// rows); rows of S evolve independently, so slices never communicate. The
-// fp32 master state lives in registers (thread t holds column t of the
-// slice); a bf16 copy in shared memory feeds the MMAs.
+// One CTA of 256 threads owns one (sequence, value head, slice of DVP state
+// rows); rows of S evolve independently, so slices never communicate. Warps
+// w and w+4 read the same TMEM lane quarter and split every row epilogue by
+// column halves. The fp32 master state lives in registers (thread (q, h)
+// holds half h of column 32q+lane of the slice); a bf16 copy in shared memory
+// (MN-major, one 16-byte-chunked row per d_k index) feeds the MMAs.
+//
+// exp(G_r - G_s) is formed as exp(G_r - m) * exp(m - G_s) with m the middle
+// of the chunk's decay range, i.e. one exponential per token instead of one
+// per matrix entry; chunks whose decay range could leave the fp32 exponent
+// range (more than e^160 across the chunk) take an exact per-entry path.
 #pragma once
 
 #include "common.cuh"
@@ -45,7 +52,7 @@ namespace tc {
 
 constexpr int kC = 64;     // chunk length
 constexpr int kD = 128;    // d_k = d_v
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
 constexpr uint32_t kTmemCols = 512;
 
 // TMEM column map (fp32 columns)
@@ -76,8 +83,8 @@ struct Smem {
   static constexpr uint32_t kUBytes = DVP * 128 < 1024 ? 1024 : DVP * 128;
   static constexpr uint32_t kUsb = kUb + kUBytes;          // U_s^T [DVP][64]
   static constexpr uint32_t kAd = kUsb + kUBytes;          // 4 diagonal blocks of A, fp32 [4][16][16]
-  static constexpr uint32_t kVec = kAd + 4 * 16 * 16 * 4;  // G, beta, rk, rq, scan scratch
-  static constexpr uint32_t kBar = kVec + 5 * 64 * 4;      // mbarriers: tma[2], mma
+  static constexpr uint32_t kVec = kAd + 4 * 16 * 16 * 4;  // G, beta, rk, rq, ck, cw, scan scratch
+  static constexpr uint32_t kBar = kVec + 7 * 64 * 4;      // mbarriers: tma[2], mma
   static constexpr uint32_t kTmemSlot = kBar + 3 * 8;
   static constexpr uint32_t kFlags = kTmemSlot + 8;
   static constexpr uint32_t kTotal = kFlags + 16;
@@ -120,14 +127,18 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
                   __nv_bfloat16* __restrict__ o, float* state_out, int total_T) {
   using L = Smem<DVP>;
   using namespace sm100;
+  constexpr int kHalf = DVP / 2;          // state-slice columns per thread
+  constexpr uint32_t kR = DVP * 2;        // bytes per row of the MN-major v / U / S tiles
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(sm);
-  float* vG = reinterpret_cast<float*>(sm + L::kVec);       // [64] cumulative log-decay
+  float* vG = reinterpret_cast<float*>(sm + L::kVec);       // [64] cumulative log-decay G
   float* vB = vG + 64;                                      // [64] beta
   float* vRk = vB + 64;                                     // [64] 1/|k|
   float* vRq = vRk + 64;                                    // [64] scale/|q|
-  float* vScan = vRq + 64;                                  // scan scratch
+  float* vCk = vRq + 64;                                    // [64] column factor of A and P
+  float* vCw = vCk + 64;                                    // [64] -beta gamma rk (column factor of T_w)
+  float* vScan = vCw + 64;                                  // scan scratch / flags
   uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + L::kBar);
   uint64_t* bar_mma = bar_tma + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kTmemSlot);
@@ -137,6 +148,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
   const int hq = h / (Hv / Hqk);
   const int i0 = part * DVP;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qd = warp & 3;                 // TMEM lane quarter
+  const int ch = warp >> 2;                // column half
+  const int r128 = qd * 32 + lane;         // row of an M=128 accumulator held by this thread
+  const int r64 = qd * 16 + (lane & 15);   // row of an M=64 accumulator (lanes 0-15 / 16-31 halves)
+  const bool lo16 = lane < 16;
 
   int t_begin = cu_seqlens[n], t_end = cu_seqlens[n + 1];
   t_end = min(t_end, total_T);
@@ -160,16 +176,20 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tlane = static_cast<uint32_t>(warp * 32) << 16;   // this warp's TMEM lane quarter
+  const uint32_t tlane = static_cast<uint32_t>(qd * 32) << 16;
 
-  // fp32 master state: thread t holds S[i0 + i][t], i < DVP
-  const size_t s_off = ((size_t)n * Hv + h) * kD * kD + (size_t)i0 * kD;
-  float Sreg[DVP];
+  // fp32 master state: S[i0 + ch*kHalf + j][r128], j < kHalf
+  const size_t s_off = ((size_t)n * Hv + h) * kD * kD + (size_t)(i0 + ch * kHalf) * kD + r128;
+  float Sreg[kHalf];
 #pragma unroll
-  for (int i = 0; i < DVP; ++i) Sreg[i] = state_in ? state_in[s_off + (size_t)i * kD + tid] : 0.f;
+  for (int j = 0; j < kHalf; ++j) Sreg[j] = state_in ? state_in[s_off + (size_t)j * kD] : 0.f;
   const uint32_t sSb = sbase + L::kSb;
+  auto store_state = [&]() {
 #pragma unroll
-  for (int i = 0; i < DVP; ++i) st_shared_b16(sSb + sw128_off(i, tid, DVP * 128), __float2bfloat16_rn(Sreg[i]));
+    for (int c = 0; c < kHalf / 8; ++c)
+      st_shared_v4(sSb + mn_off<kR>(r128, ch * kHalf + 8 * c), pack8_bf16(Sreg + 8 * c));
+  };
+  store_state();
 
   auto issue_tma = [&](int ci) {
     const int slot = ci & 1;
@@ -187,11 +207,20 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     if (nchunks > 1) issue_tma(1);
   }
 
+  // gates of the next chunk are fetched one chunk ahead (threads 0-63)
+  float g_next = 0.f, b_next = 0.f;
+  auto fetch_gates = [&](int ci) {
+    const int c0 = t_begin + ci * kC;
+    const bool valid = ci < nchunks && c0 + tid < t_end;
+    g_next = valid ? g[(size_t)(c0 + tid) * Hv + h] : 0.f;
+    b_next = valid ? beta[(size_t)(c0 + tid) * Hv + h] : 0.f;
+  };
+  if (tid < 64) fetch_gates(0);
+
   uint32_t mma_phase = 0;
   uint32_t tma_phase[2] = {0, 0};
   bool abort = false;
 
-  // Wait for the MMA barrier; a timeout anywhere aborts the whole CTA.
   auto wait_mma = [&]() -> bool {
     bool ok = mbar_wait(bar_mma, mma_phase);
     mma_phase ^= 1;
@@ -199,7 +228,6 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     tc_fence_after();
     return ok;
   };
-  // Make this thread's shared-memory and TMEM reads/writes visible before an MMA issue.
   auto publish = [&]() {
     fence_async_smem();
     tc_fence_before();
@@ -210,10 +238,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
   constexpr uint32_t kIdG = idesc_bf16(128, 128, false, false);
   constexpr uint32_t kId64 = idesc_bf16(64, 64, false, true);      // K-major A, MN-major B
   constexpr uint32_t kIdW = idesc_bf16(64, 128, false, true);
-  constexpr uint32_t kIdU = idesc_bf16(64, DVP, false, true);
-  constexpr uint32_t kIdChain = idesc_bf16(64, DVP, false, false);
-  constexpr uint32_t kIdDS = idesc_bf16(128, DVP, true, false);
-  constexpr uint32_t kVRow = DVP * 2;   // bytes per v row (swizzle width)
+  constexpr uint32_t kIdSlice = idesc_bf16(64, DVP, false, true);
+  constexpr uint32_t kIdDS = idesc_bf16(128, DVP, true, true);
 
   for (int ci = 0; ci < nchunks && !abort; ++ci) {
     const int slot = ci & 1;
@@ -222,19 +248,21 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     const uint32_t sKQ = sbase + L::kKQ + slot * L::kKQBytes;
     const uint32_t sV = sbase + L::kV + slot * L::kVStride;
 
-    // ---- gates: cumulative log-decay and beta (rows >= Lc are padding) ----
+    // ---- gates: inclusive scan of g, beta; next chunk's gates prefetched ----
     if (tid < 64) {
-      const bool valid = tid < Lc;
-      float gv = valid ? g[(size_t)(c0 + tid) * Hv + h] : 0.f;
-      const float bv = valid ? beta[(size_t)(c0 + tid) * Hv + h] : 0.f;
+      float gv = g_next;
+      const float bv = b_next;
+      const unsigned nonpos = __ballot_sync(0xffffffffu, gv <= 0.f);
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
         const float up = __shfl_up_sync(0xffffffffu, gv, off);
         if (lane >= off) gv += up;
       }
       if (lane == 31) vScan[warp] = gv;
+      if (lane == 0) vScan[2 + warp] = nonpos == 0xffffffffu ? 1.f : 0.f;
       vB[tid] = bv;
       vG[tid] = gv;
+      fetch_gates(ci + 1);
     }
     {
       bool ok = mbar_wait(&bar_tma[slot], tma_phase[slot]);
@@ -243,7 +271,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     }
     if (tid >= 32 && tid < 64) vG[tid] += vScan[0];
 
-    // ---- [k;q][k;q]^T : KK^T (rows 0-63), QK^T (rows 64-127), norms on the diagonal ----
+    // ---- [k;q][k;q]^T : KK^T (rows 0-63), QK^T (rows 64-127), squared norms on the diagonal ----
     if (tid == 0) {
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
@@ -252,86 +280,123 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     }
     if (!wait_mma()) { abort = true; break; }
 
-    float row[64];
+    const float G0 = vG[0], GL = vG[Lc - 1];
+    const bool fast = vScan[2] > 0.f && vScan[3] > 0.f && (G0 - GL) <= 160.f;
+    const float gm = 0.5f * (G0 + GL);   // reference point of the factored decay
+
+    float rowv[32];   // columns 32ch..32ch+31 of row r128
+    tmem_ld32(tmem + tlane + kColG + 32 * ch, rowv);
     {
-      float tmp[32];
-      tmem_ld32(tmem + tlane + kColG, tmp);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) row[j] = tmp[j];
-      tmem_ld32(tmem + tlane + kColG + 32, tmp);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) row[32 + j] = tmp[j];
-      // own squared norm: column tid of row tid
+      bool own = false;
       float diag = 0.f;
-      if (warp < 2) {
+      if (qd < 2) {
+        own = (qd == ch);
 #pragma unroll
-        for (int j = 0; j < 64; ++j) diag = (j == tid) ? row[j] : diag;
-      } else {
-        tmem_ld32(tmem + tlane + kColG + 64 + 32 * (warp - 2), tmp);
+        for (int j = 0; j < 32; ++j) diag = (j == lane) ? rowv[j] : diag;
+      } else if (ch == 0) {
+        float tmp[32];
+        tmem_ld32(tmem + tlane + kColG + 64 + 32 * (qd - 2), tmp);
 #pragma unroll
         for (int j = 0; j < 32; ++j) diag = (j == lane) ? tmp[j] : diag;
+        own = true;
       }
-      const int r = tid & 63;
-      const bool valid = r < Lc;
-      if (tid < 64) vRk[r] = valid ? 1.0f / sqrtf(diag + kNormEps) : 0.f;
-      else vRq[r] = valid ? scale / sqrtf(diag + kNormEps) : 0.f;
+      if (own) {
+        const int r = r128 & 63;
+        const bool valid = r < Lc;
+        if (qd < 2) {
+          const float rk = valid ? 1.0f / sqrtf(diag + kNormEps) : 0.f;
+          const float Gr = vG[r];
+          vRk[r] = rk;
+          vCk[r] = fast ? expf(gm - Gr) * rk : rk;
+          vCw[r] = -vB[r] * expf(Gr) * rk;
+        } else {
+          vRq[r] = valid ? scale / sqrtf(diag + kNormEps) : 0.f;
+        }
+      }
     }
     __syncthreads();
 
-    // ---- A (diagonal blocks fp32, off-diagonal blocks bf16) and P ----
+    // ---- A (diagonal blocks fp32, off-diagonal blocks bf16) and P, half a row per thread ----
     {
-      const int r = tid & 63;
+      const int r = r128 & 63;
       const float Gr = vG[r];
-      if (tid < 64) {
-        const float fr = vB[r] * vRk[r];
-        const int b = r >> 4;
-        float a[64];
+      float x[32];
+      if (qd < 2) {
+        const float fr = vB[r] * vRk[r] * (fast ? expf(Gr - gm) : 1.f);
+        if (fast) {
 #pragma unroll
-        for (int s = 0; s < 64; ++s) a[s] = (s < r) ? fr * vRk[s] * expf(Gr - vG[s]) * row[s] : 0.f;
-        // diagonal block (fp32, for the forward substitution)
+          for (int j = 0; j < 32; ++j) {
+            const int s = 32 * ch + j;
+            x[j] = (s < r) ? fr * vCk[s] * rowv[j] : 0.f;
+          }
+        } else {
 #pragma unroll
-        for (int bb = 0; bb < 4; ++bb) {
-          if (bb == b) {
-#pragma unroll
-            for (int s = 0; s < 16; ++s) Ad[(bb * 16 + (r & 15)) * 16 + s] = a[bb * 16 + s];
+          for (int j = 0; j < 32; ++j) {
+            const int s = 32 * ch + j;
+            x[j] = (s < r) ? fr * vCk[s] * expf(Gr - vG[s]) * rowv[j] : 0.f;
           }
         }
-        // A_o: blocks strictly left of the diagonal block
-        float ao[64];
+        const int b = r >> 4;
+        if ((b >> 1) == ch) {   // this half holds the diagonal block: keep it in fp32
+          float* dst = Ad + (b * 16 + (r & 15)) * 16;
+          if (b & 1) {
 #pragma unroll
-        for (int s = 0; s < 64; ++s) ao[s] = (s < 16 * b) ? a[s] : 0.f;
-        store_row64(sbase + L::kAo, r, ao);
+            for (int j = 0; j < 16; ++j) dst[j] = x[16 + j];
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) dst[j] = x[j];
+          }
+        }
+        // A_o: only the blocks strictly left of the diagonal block
+#pragma unroll
+        for (int j = 0; j < 32; ++j) x[j] = (32 * ch + j < 16 * b) ? x[j] : 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          st_shared_v4(sbase + L::kAo + sw128_off(r, 32 * ch + 8 * c, 0), pack8_bf16(x + 8 * c));
       } else {
-        const float fr = vRq[r];
-        float p[64];
+        const float fr = vRq[r] * (fast ? expf(Gr - gm) : 1.f);
+        if (fast) {
 #pragma unroll
-        for (int s = 0; s < 64; ++s) p[s] = (s <= r) ? fr * vRk[s] * expf(Gr - vG[s]) * row[s] : 0.f;
-        store_row64(sbase + L::kPm, r, p);
+          for (int j = 0; j < 32; ++j) {
+            const int s = 32 * ch + j;
+            x[j] = (s <= r) ? fr * vCk[s] * rowv[j] : 0.f;
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int s = 32 * ch + j;
+            x[j] = (s <= r) ? fr * vCk[s] * expf(Gr - vG[s]) * rowv[j] : 0.f;
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          st_shared_v4(sbase + L::kPm + sw128_off(r, 32 * ch + 8 * c, 0), pack8_bf16(x + 8 * c));
       }
     }
     __syncthreads();
 
-    // ---- D = (I + A_d)^-1, one column of one diagonal block per thread ----
+    // ---- D = (I + A_d)^-1: one column of one diagonal block per thread (threads 0-63) ----
     if (tid < 64) {
       const int b = tid >> 4, j = tid & 15;
       const float* Ab = Ad + b * 256;
-      float x[16];
+      float xs[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         float acc = 0.f;
 #pragma unroll
-        for (int k2 = 0; k2 < i; ++k2) acc = fmaf(Ab[i * 16 + k2], x[k2], acc);
-        x[i] = (i == j) ? 1.f : (i > j ? -acc : 0.f);
+        for (int k2 = 0; k2 < i; ++k2) acc = fmaf(Ab[i * 16 + k2], xs[k2], acc);
+        xs[i] = (i == j) ? 1.f : (i > j ? -acc : 0.f);
       }
 #pragma unroll
       for (int i = 0; i < 16; ++i)
-        st_shared_b16(sbase + L::kDm + sw128_off(16 * b + i, 16 * b + j, 0), __float2bfloat16_rn(x[i]));
+        st_shared_b16(sbase + L::kDm + sw128_off(16 * b + i, 16 * b + j, 0), __float2bfloat16_rn(xs[i]));
     } else {
-      // zero the off-diagonal blocks of D
-      const int r = tid - 64, b = r >> 4;
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        if ((c >> 1) != b) st_shared_v4(sbase + L::kDm + sw128_off(r, 8 * c, 0), make_uint4(0, 0, 0, 0));
+      // zero the off-diagonal blocks of D: 64 rows x 6 chunks
+      for (int e = tid - 64; e < 64 * 6; e += kThreads - 64) {
+        const int row = e / 6, idx = e - row * 6, b = row >> 4;
+        const int c = idx < 2 * b ? idx : idx + 2;
+        st_shared_v4(sbase + L::kDm + sw128_off(row, 8 * c, 0), make_uint4(0, 0, 0, 0));
+      }
     }
     publish();
 
@@ -345,15 +410,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     }
     if (!wait_mma()) { abort = true; break; }
     {
-      float tmp[32];
-      float v[64];
-      tmem_ld32(tmem + tlane + kColN, tmp);
+      float v[32];
+      tmem_ld32(tmem + tlane + kColN + 32 * ch, v);
+      if (lo16) {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = tmp[j];
-      tmem_ld32(tmem + tlane + kColN + 32, tmp);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) v[32 + j] = tmp[j];
-      if (lane < 16) store_row64(sbase + L::kNm, warp * 16 + lane, v);
+        for (int c = 0; c < 4; ++c)
+          st_shared_v4(sbase + L::kNm + sw128_off(r64, 32 * ch + 8 * c, 0), pack8_bf16(v + 8 * c));
+      }
     }
     publish();
 
@@ -370,21 +433,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       mma_commit(bar_mma);
     }
     if (!wait_mma()) { abort = true; break; }
-    float E[64];   // lanes 0-15: row of E = D - N D (fp32)
+    float E[32];   // lanes 0-15: half row of E = D - N D (fp32)
     {
-      float tmp[32];
-      tmem_ld32(tmem + tlane + kColN, tmp);
+      tmem_ld32(tmem + tlane + kColN + 32 * ch, E);
+      if (lo16) {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) E[j] = tmp[j];
-      tmem_ld32(tmem + tlane + kColN + 32, tmp);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) E[32 + j] = tmp[j];
-      const int r = warp * 16 + (lane & 15);
-      if (lane < 16) {
-        // E = D - N D, with D read back from its bf16 tile
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 dv = ld_shared_v4(sbase + L::kDm + sw128_off(r, 8 * c, 0));
+        for (int c = 0; c < 4; ++c) {
+          const uint4 dv = ld_shared_v4(sbase + L::kDm + sw128_off(r64, 32 * ch + 8 * c, 0));
           const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -392,10 +447,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             E[8 * c + 2 * e] = df.x - E[8 * c + 2 * e];
             E[8 * c + 2 * e + 1] = df.y - E[8 * c + 2 * e + 1];
           }
+          st_shared_v4(sbase + L::kEm + sw128_off(r64, 32 * ch + 8 * c, 0), pack8_bf16(E + 8 * c));
         }
-        store_row64(sbase + L::kEm, r, E);
       } else {
-        store_row64(sbase + L::kAo, r, E);   // N^2 (A_o no longer needed)
+#pragma unroll
+        for (int c = 0; c < 4; ++c)   // N^2 (A_o is no longer needed)
+          st_shared_v4(sbase + L::kAo + sw128_off(r64, 32 * ch + 8 * c, 0), pack8_bf16(E + 8 * c));
       }
     }
     publish();
@@ -410,29 +467,26 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     }
     if (!wait_mma()) { abort = true; break; }
     {
-      float tmp[32];
-      float tw[64], tu[64];
+      float z[32], tw[32], tu[32];
+      tmem_ld32(tmem + tlane + kColZ + 32 * ch, z);
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        tmem_ld32(tmem + tlane + kColZ + 32 * half, tmp);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int s = 32 * half + j;
-          const float t = E[s] + tmp[j];
-          const float bs = vB[s];
-          tu[s] = t * bs;
-          tw[s] = t * bs * expf(vG[s]) * vRk[s];
-        }
+      for (int j = 0; j < 32; ++j) {
+        const int s = 32 * ch + j;
+        const float t = E[j] + z[j];
+        tu[j] = t * vB[s];
+        tw[j] = t * vCw[s];   // carries the minus sign: the MMA below yields -W
       }
-      if (lane < 16) {
-        const int r = warp * 16 + lane;
-        store_row64(sbase + L::kNm, r, tw);   // T_w (N no longer needed)
-        store_row64(sbase + L::kEm, r, tu);   // T_u (E no longer needed)
+      if (lo16) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          st_shared_v4(sbase + L::kNm + sw128_off(r64, 32 * ch + 8 * c, 0), pack8_bf16(tw + 8 * c));
+          st_shared_v4(sbase + L::kEm + sw128_off(r64, 32 * ch + 8 * c, 0), pack8_bf16(tu + 8 * c));
+        }
       }
     }
     publish();
 
-    // ---- W = T_w K_raw  (M=64, N=128) ;  U~ = T_u V_raw (M=64, N=DVP) ----
+    // ---- -W = -T_w K_raw  (M=64, N=128) ;  U~ = T_u V_raw (M=64, N=DVP) ----
     if (tid == 0) {
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
@@ -440,26 +494,19 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
                  kk > 0);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + kColU, desc_kmajor(sbase + L::kEm, kk, 0), desc_mnmajor(sV, kk, kVRow, L::kVBytes),
-                 kIdU, kk > 0);
+        mma_bf16(tmem + kColU, desc_kmajor(sbase + L::kEm, kk, 0), desc_mnmajor(sV, kk, kR, L::kVBytes),
+                 kIdSlice, kk > 0);
       mma_commit(bar_mma);
     }
     if (!wait_mma()) { abort = true; break; }
     {
-      float tmp[32];
+      float w[64];
+      tmem_ld32(tmem + tlane + kColW + 64 * ch, w);
+      tmem_ld32(tmem + tlane + kColW + 64 * ch + 32, w + 32);
+      if (lo16) {
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        tmem_ld32(tmem + tlane + kColW + 32 * q4, tmp);
-        if (lane < 16) {
-          const int r = warp * 16 + lane;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            float x[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] = -tmp[8 * c + e];
-            st_shared_v4(sbase + L::kWn + sw128_off(r, 32 * q4 + 8 * c, 8192), pack8_bf16(x));
-          }
-        }
+        for (int c = 0; c < 8; ++c)
+          st_shared_v4(sbase + L::kWn + sw128_off(r64, 64 * ch + 8 * c, 8192), pack8_bf16(w + 8 * c));
       }
     }
     publish();
@@ -468,42 +515,33 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     if (tid == 0) {
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
-        mma_bf16(tmem + kColU, desc_kmajor(sbase + L::kWn, kk, 8192), desc_kmajor(sSb, kk, DVP * 128),
-                 kIdChain, 1);
+        mma_bf16(tmem + kColU, desc_kmajor(sbase + L::kWn, kk, 8192), desc_mnmajor(sSb, kk, kR, 128 * kR),
+                 kIdSlice, 1);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
         mma_bf16(tmem + (16u << 16) + kColU, desc_kmajor(sKQ + 8192, kk, 16384),
-                 desc_kmajor(sSb, kk, DVP * 128), kIdChain, kk > 0);
+                 desc_mnmajor(sSb, kk, kR, 128 * kR), kIdSlice, kk > 0);
       mma_commit(bar_mma);
     }
     if (!wait_mma()) { abort = true; break; }
-    const float GL = vG[Lc - 1];
-    float oq[DVP];   // lanes 16-31: gamma_r rq_r (Q_raw S^T)_r
+    float oq[kHalf];   // lanes 16-31: gamma_r rq_r (Q_raw S^T)_r, this thread's column half
     {
-      float uv[DVP];
-      if constexpr (DVP == 16) {
-        tmem_ld16(tmem + tlane + kColU, uv);
-      } else {
+      float uv[kHalf];
+      tmem_ld<kHalf>(tmem + tlane + kColU + ch * kHalf, uv);
+      if (lo16) {
+        const float us = expf(GL - vG[r64]) * vRk[r64];
+        float usv[kHalf];
 #pragma unroll
-        for (int q32 = 0; q32 < DVP / 32; ++q32) {
-          float tmp[32];
-          tmem_ld32(tmem + tlane + kColU + 32 * q32, tmp);
+        for (int j = 0; j < kHalf; ++j) usv[j] = uv[j] * us;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) uv[32 * q32 + j] = tmp[j];
-        }
-      }
-      const int r = warp * 16 + (lane & 15);
-      if (lane < 16) {
-        const float us = expf(GL - vG[r]) * vRk[r];
-#pragma unroll
-        for (int i = 0; i < DVP; ++i) {
-          st_shared_b16(sbase + L::kUb + sw128_off(i, r, 0), __float2bfloat16_rn(uv[i]));
-          st_shared_b16(sbase + L::kUsb + sw128_off(i, r, 0), __float2bfloat16_rn(uv[i] * us));
+        for (int c = 0; c < kHalf / 8; ++c) {
+          st_shared_v4(sbase + L::kUb + mn_off<kR>(r64, ch * kHalf + 8 * c), pack8_bf16(uv + 8 * c));
+          st_shared_v4(sbase + L::kUsb + mn_off<kR>(r64, ch * kHalf + 8 * c), pack8_bf16(usv + 8 * c));
         }
       } else {
-        const float rho = expf(vG[r]) * vRq[r];
+        const float rho = expf(vG[r64]) * vRq[r64];
 #pragma unroll
-        for (int i = 0; i < DVP; ++i) oq[i] = rho * uv[i];
+        for (int j = 0; j < kHalf; ++j) oq[j] = rho * uv[j];
       }
     }
     publish();
@@ -513,50 +551,32 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
         mma_bf16(tmem + (16u << 16) + kColPU, desc_kmajor(sbase + L::kPm, kk, 0),
-                 desc_kmajor(sbase + L::kUb, kk, 0), kIdChain, kk > 0);
+                 desc_mnmajor(sbase + L::kUb, kk, kR, 64 * kR), kIdSlice, kk > 0);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + kColDS, desc_mnmajor(sKQ, kk, 128, 16384), desc_kmajor(sbase + L::kUsb, kk, 0),
+        mma_bf16(tmem + kColDS, desc_mnmajor(sKQ, kk, 128, 16384), desc_mnmajor(sbase + L::kUsb, kk, kR, 64 * kR),
                  kIdDS, kk > 0);
       mma_commit(bar_mma);
     }
     if (!wait_mma()) { abort = true; break; }
     {
-      float pu[DVP], ds[DVP];
-      if constexpr (DVP == 16) {
-        tmem_ld16(tmem + tlane + kColPU, pu);
-        tmem_ld16(tmem + tlane + kColDS, ds);
-      } else {
+      float pu[kHalf], ds[kHalf];
+      tmem_ld<kHalf>(tmem + tlane + kColPU + ch * kHalf, pu);
+      tmem_ld<kHalf>(tmem + tlane + kColDS + ch * kHalf, ds);
+      if (!lo16 && r64 < Lc) {
+        __nv_bfloat16* orow = o + ((size_t)(c0 + r64) * Hv + h) * kD + i0 + ch * kHalf;
 #pragma unroll
-        for (int q32 = 0; q32 < DVP / 32; ++q32) {
-          float tmp[32];
-          tmem_ld32(tmem + tlane + kColPU + 32 * q32, tmp);
+        for (int c = 0; c < kHalf / 8; ++c) {
+          float xo[8];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) pu[32 * q32 + j] = tmp[j];
-          tmem_ld32(tmem + tlane + kColDS + 32 * q32, tmp);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) ds[32 * q32 + j] = tmp[j];
-        }
-      }
-      if (lane >= 16) {
-        const int r = warp * 16 + lane - 16;
-        if (r < Lc) {
-          __nv_bfloat16* orow = o + ((size_t)(c0 + r) * Hv + h) * kD + i0;
-#pragma unroll
-          for (int c = 0; c < DVP / 8; ++c) {
-            float x[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] = oq[8 * c + e] + pu[8 * c + e];
-            *reinterpret_cast<uint4*>(orow + 8 * c) = pack8_bf16(x);
-          }
+          for (int e = 0; e < 8; ++e) xo[e] = oq[8 * c + e] + pu[8 * c + e];
+          *reinterpret_cast<uint4*>(orow + 8 * c) = pack8_bf16(xo);
         }
       }
       const float gL = expf(GL);
 #pragma unroll
-      for (int i = 0; i < DVP; ++i) {
-        Sreg[i] = fmaf(gL, Sreg[i], ds[i]);
-        st_shared_b16(sSb + sw128_off(i, tid, DVP * 128), __float2bfloat16_rn(Sreg[i]));
-      }
+      for (int j = 0; j < kHalf; ++j) Sreg[j] = fmaf(gL, Sreg[j], ds[j]);
+      store_state();
     }
     publish();
     // the raw tiles of this slot are free (every MMA reading them completed)
@@ -571,7 +591,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     __syncthreads();
   } else {
 #pragma unroll
-    for (int i = 0; i < DVP; ++i) state_out[s_off + (size_t)i * kD + tid] = Sreg[i];
+    for (int j = 0; j < kHalf; ++j) state_out[s_off + (size_t)j * kD] = Sreg[j];
   }
   tc_fence_before();
   __syncthreads();

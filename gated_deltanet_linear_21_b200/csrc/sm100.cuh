@@ -162,9 +162,32 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int col, uint32_t acs) {
          ((((col & 63) >> 3) ^ (row & 7)) << 4) + ((col & 7) << 1);
 }
 
+// Byte offset of element (row, col) of an MN-major tile whose rows are R
+// bytes (32, 64 or 128) with the matching swizzle: 16-byte chunk bits [4,7)
+// XOR address bits [7,10) (as many bits as the row has chunks).
+template <uint32_t R>
+__device__ __forceinline__ uint32_t mn_off(int row, int col) {
+  static_assert(R == 32 || R == 64 || R == 128, "row bytes");
+  constexpr uint32_t mask = R == 128 ? 7u : R == 64 ? 3u : 1u;
+  const uint32_t o = static_cast<uint32_t>(row) * R + static_cast<uint32_t>(col) * 2u;
+  return o ^ (((o >> 7) & mask) << 4);
+}
+
 // ------------------------------------------------------------ TMEM loads ---
-// 32 lanes x 16 / 32 consecutive 32-bit columns, waited for before returning.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&r)[16]) {
+// 32 lanes x 8 / 16 / 32 consecutive 32-bit columns, waited for before returning.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* r) {
+  uint32_t u[8];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i) r[i] = __uint_as_float(u[i]);
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* r) {
   uint32_t u[16];
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
@@ -179,7 +202,7 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&r)[16]) {
   for (int i = 0; i < 16; ++i) r[i] = __uint_as_float(u[i]);
 }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32]) {
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* r) {
   uint32_t u[32];
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
@@ -195,6 +218,20 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32]) {
       : "memory");
 #pragma unroll
   for (int i = 0; i < 32; ++i) r[i] = __uint_as_float(u[i]);
+}
+
+// Load N (8, 16, 32 or a multiple of 32) consecutive columns.
+template <int N>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, float* r) {
+  if constexpr (N == 8) {
+    tmem_ld8(taddr, r);
+  } else if constexpr (N == 16) {
+    tmem_ld16(taddr, r);
+  } else {
+    static_assert(N % 32 == 0, "columns");
+#pragma unroll
+    for (int c = 0; c < N / 32; ++c) tmem_ld32(taddr + 32 * c, r + 32 * c);
+  }
 }
 
 // Pack 8 floats into 8 bf16 (round to nearest even) as one 16-byte chunk.
