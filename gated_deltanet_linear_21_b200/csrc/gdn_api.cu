@@ -157,12 +157,10 @@ bool make_map(CUtensorMap* m, const void* base, int D, int H, int T, int box_d) 
 int tc_slice_rows(int n_seqs, int Hv) {
   if (const char* env = getenv("GDN_TC_SLICE")) {
     const int v = atoi(env);
-    if (v == 16 || v == 32 || v == 64) return v;
+    if (v == 16 || v == 32) return v;
   }
   const long chains = (long)n_seqs * Hv;
-  if (chains <= 18) return 16;
-  if (chains <= 37) return 32;
-  return 64;
+  return chains <= 18 ? 16 : 32;
 }
 
 template <int DVP>
@@ -186,11 +184,9 @@ gdn_status launch_prefill_tc(const void* q, const void* k, const void* v, const 
   if (!make_map(&qm, q, 128, Hqk, (int)total_T, 64) || !make_map(&km, k, 128, Hqk, (int)total_T, 64) ||
       !make_map(&vm, v, 128, Hv, (int)total_T, dvp))
     return fail(GDN_ERR_CUDA, "gdn_prefill: cuTensorMapEncodeTiled unavailable or failed");
-  switch (dvp) {
-    case 16: return launch_tc<16>(qm, km, vm, g, beta, state_in, cu, n_seqs, Hqk, Hv, scale, o, state_out, (int)total_T, st);
-    case 32: return launch_tc<32>(qm, km, vm, g, beta, state_in, cu, n_seqs, Hqk, Hv, scale, o, state_out, (int)total_T, st);
-    default: return launch_tc<64>(qm, km, vm, g, beta, state_in, cu, n_seqs, Hqk, Hv, scale, o, state_out, (int)total_T, st);
-  }
+  if (dvp == 16)
+    return launch_tc<16>(qm, km, vm, g, beta, state_in, cu, n_seqs, Hqk, Hv, scale, o, state_out, (int)total_T, st);
+  return launch_tc<32>(qm, km, vm, g, beta, state_in, cu, n_seqs, Hqk, Hv, scale, o, state_out, (int)total_T, st);
 }
 
 }  // namespace
