@@ -6,6 +6,7 @@
 #include <mutex>
 #include <set>
 #include <string>
+#include <algorithm>
 #include <utility>
 
 #include "gdn.h"
@@ -13,6 +14,7 @@
 #include "decode.cuh"
 #include "prefill_simt.cuh"
 #include "prefill_tc.cuh"
+#include "prefill_pc.cuh"
 
 #include <cudaTypedefs.h>
 #include <cstdlib>
@@ -176,6 +178,80 @@ gdn_status launch_tc(const CUtensorMap& qm, const CUtensorMap& km, const CUtenso
   return launch_status("gdn_prefill");
 }
 
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+bool uses_pc_prefill(gdn_dtype dtype, int dk, int dv) {
+  return dtype == GDN_BF16 && dk == 128 && dv == 128 && !getenv("GDN_PREFILL_FUSED");
+}
+
+template <int DVP>
+gdn_status launch_pc(const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm,
+                     const gdn::pc::Params& prm, int grid, cudaStream_t st) {
+  auto kern = gdn::pc::prefill_pc_kernel<DVP>;
+  if (gdn_status s = allow_smem(kern, "gdn_prefill")) return s;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(gdn::pc::kThreads);
+  cfg.dynamicSmemBytes = gdn::pc::Smem<DVP>::kAlloc;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;   // every CTA co-resident: CTAs wait on one another
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, qm, km, vm, prm);
+  if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "gdn_prefill: launch failed: %s", cudaGetErrorString(e));
+  return launch_status("gdn_prefill");
+}
+
+gdn_status launch_prefill_pc(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                             const float* state_in, const int32_t* cu, int n_seqs, int64_t total_T, int Hqk,
+                             int Hv, float scale, void* o, float* state_out, void* ws, cudaStream_t st) {
+  const long chains = (long)n_seqs * Hv;
+  const int sms = sm_count();
+  if (sms < 4) return fail(GDN_ERR_CUDA, "gdn_prefill: cannot query the multiprocessor count");
+  int dvp = chains * 4 <= (long)(sms * 0.45) ? 32 : 64;
+  if (const char* env = getenv("GDN_TC_SLICE")) {
+    const int v2 = atoi(env);
+    if (v2 == 32 || v2 == 64) dvp = v2;
+  }
+  const int slices = 128 / dvp;
+  long nc = (long)(sms * 0.45);
+  nc = std::min(nc, chains * slices);
+  nc -= nc % slices;
+  if (nc < slices) nc = slices;
+  const long rounds = (chains * slices + nc - 1) / nc;
+  if (rounds > gdn::pc::kMaxRounds)
+    return fail(GDN_ERR_UNSUPPORTED, "gdn_prefill: %ld sequence-heads is more than this kernel schedules", chains);
+  CUtensorMap qm, km, vm;
+  if (!make_map(&qm, q, 128, Hqk, (int)total_T, 64) || !make_map(&km, k, 128, Hqk, (int)total_T, 64) ||
+      !make_map(&vm, v, 128, Hv, (int)total_T, dvp))
+    return fail(GDN_ERR_CUDA, "gdn_prefill: cuTensorMapEncodeTiled unavailable or failed");
+  cudaError_t e = cudaMemsetAsync(ws, 0, gdn::pc::Workspace::zeroed_bytes(chains), st);
+  if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "gdn_prefill: %s", cudaGetErrorString(e));
+  gdn::pc::Params prm;
+  prm.g = g;
+  prm.beta = beta;
+  prm.state_in = state_in;
+  prm.cu_seqlens = cu;
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.state_out = state_out;
+  prm.ws = static_cast<uint8_t*>(ws);
+  prm.n_seqs = n_seqs;
+  prm.Hqk = Hqk;
+  prm.Hv = Hv;
+  prm.total_T = (int)total_T;
+  prm.scale = scale;
+  prm.n_chain_ctas = (int)nc;
+  if (dvp == 32) return launch_pc<32>(qm, km, vm, prm, sms, st);
+  return launch_pc<64>(qm, km, vm, prm, sms, st);
+}
+
 gdn_status launch_prefill_tc(const void* q, const void* k, const void* v, const float* g, const float* beta,
                              const float* state_in, const int32_t* cu, int n_seqs, int64_t total_T, int Hqk,
                              int Hv, float scale, void* o, float* state_out, cudaStream_t st) {
@@ -198,8 +274,8 @@ int gdn_version(void) { return (0 << 16) | 1; }
 const char* gdn_last_error(void) { return t_last_error.c_str(); }
 
 size_t gdn_prefill_workspace_bytes(int n_seqs, int Hv, int dk, int dv, gdn_dtype dtype) {
-  (void)n_seqs; (void)Hv; (void)dk; (void)dv; (void)dtype;
-  return 0;
+  if (n_seqs <= 0 || Hv <= 0 || !uses_pc_prefill(dtype, dk, dv)) return 0;
+  return gdn::pc::Workspace::bytes((long)n_seqs * Hv);
 }
 
 gdn_status gdn_prefill(const void* q, const void* k, const void* v, const float* g,
@@ -226,16 +302,19 @@ gdn_status gdn_prefill(const void* q, const void* k, const void* v, const float*
     return fail(GDN_ERR_INVALID_ARG, "gdn_prefill: q, k, v, o and the states must be 16-byte aligned");
   if (!aligned4(g) || !aligned4(beta) || !aligned4(cu_seqlens))
     return fail(GDN_ERR_INVALID_ARG, "gdn_prefill: g, beta and cu_seqlens must be 4-byte aligned");
-  const size_t need = gdn_prefill_workspace_bytes(n_seqs, Hv, dk, dv, dtype);
-  if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace)))
-    return fail(GDN_ERR_INVALID_ARG, "gdn_prefill: workspace needs %zu bytes (16-byte aligned), got %zu",
-                need, workspace_bytes);
   if (scale <= 0.f) scale = 1.0f / sqrtf((float)dk);
   int C = chunk;
   if (C == 0) C = (dtype == GDN_BF16 && dk == 128 && dv == 128) ? 64 : 16;
   if (C != 16 && C != 32 && C != 64)
     return fail(GDN_ERR_UNSUPPORTED, "gdn_prefill: chunk=%d (supported: 16, 32, 64)", C);
+  const size_t need = gdn_prefill_workspace_bytes(n_seqs, Hv, dk, dv, dtype);
+  if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace)))
+    return fail(GDN_ERR_INVALID_ARG, "gdn_prefill: workspace needs %zu bytes (16-byte aligned), got %zu",
+                need, workspace_bytes);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (uses_pc_prefill(dtype, dk, dv) && C == 64 && total_T > 0)
+    return launch_prefill_pc(q, k, v, g, beta, state_in, cu_seqlens, n_seqs, total_T, Hqk, Hv, scale, o, state_out,
+                             workspace, st);
   if (dtype == GDN_BF16 && dk == 128 && dv == 128 && C == 64 && total_T > 0)
     return launch_prefill_tc(q, k, v, g, beta, state_in, cu_seqlens, n_seqs, total_T, Hqk, Hv, scale, o,
                              state_out, st);
