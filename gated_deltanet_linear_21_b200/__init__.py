@@ -16,7 +16,7 @@ import threading
 
 import torch
 
-__all__ = ["prefill", "decode", "prefill_workspace_bytes", "device_error", "GdnError",
+__all__ = ["prefill", "prefill_noalloc", "decode", "prefill_workspace_bytes", "device_error", "GdnError",
            "lib", "library_path", "GDN_BF16", "GDN_F32"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -47,6 +47,8 @@ SIGNATURES = {
     "gdn_prefill": (_i, [_vp, _vp, _vp, _fp, _fp, _fp, _i32p, _i, _i64, _i, _i, _i, _i, _f, _i, _i,
                          _vp, _fp, _vp, _sz, _vp]),
     "gdn_decode": (_i, [_vp, _vp, _vp, _fp, _fp, _fp, _i, _i, _i, _i, _i, _f, _i, _vp, _vp]),
+    "gdn_prefill_noalloc": (_i, [_vp, _vp, _vp, _fp, _fp, _fp, _i32p, _i, _i64, _i, _i, _i, _i, _f, _i, _i,
+                                 _vp, _fp, _vp]),
     "gdn_device_error": (_i, [_vp]),
 }
 
@@ -133,6 +135,31 @@ def prefill(q, k, v, g, beta, state_in=None, cu_seqlens=None, *, scale=None, chu
         state_in.data_ptr() if state_in is not None else None, cu_seqlens.data_ptr(),
         N, T, Hqk, Hv, dk, dv, float(scale or 0.0), int(chunk), _dtype_code(q),
         o.data_ptr(), state_out.data_ptr(), ws_ptr, ws_bytes, _stream_handle(stream)))
+    return o, state_out
+
+
+def prefill_noalloc(q, k, v, g, beta, state_in=None, cu_seqlens=None, *, scale=None, o=None,
+                    state_out=None, stream=None):
+    """gdn_prefill_noalloc: the prefill with the library's built-in scratch
+    instead of a workspace (for callers that cannot allocate device memory).
+    Outputs are allocated here only if not given."""
+    _dev(q, "q"); _dev(k, "k", q.dtype); _dev(v, "v", q.dtype)
+    _dev(g, "g", torch.float32); _dev(beta, "beta", torch.float32)
+    T, Hqk, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[2]
+    if cu_seqlens is None:
+        cu_seqlens = torch.tensor([0, T], dtype=torch.int32, device=q.device)
+    _dev(cu_seqlens, "cu_seqlens", torch.int32)
+    N = cu_seqlens.numel() - 1
+    if o is None:
+        o = torch.empty(T, Hv, dv, dtype=q.dtype, device=q.device)
+    if state_out is None:
+        state_out = torch.empty(N, Hv, dv, dk, dtype=torch.float32, device=q.device)
+    _check(lib().gdn_prefill_noalloc(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), g.data_ptr(), beta.data_ptr(),
+        state_in.data_ptr() if state_in is not None else None, cu_seqlens.data_ptr(),
+        N, T, Hqk, Hv, dk, dv, float(scale or 0.0), 0, _dtype_code(q),
+        o.data_ptr(), state_out.data_ptr(), _stream_handle(stream)))
     return o, state_out
 
 

@@ -368,3 +368,75 @@ gdn_status gdn_device_error(void* stream) {
 }
 
 }  // extern "C"
+
+// ============================================================================
+// Allocation-free prefill.
+//
+// Some callers cannot hand the library any device memory of its own making:
+// code that runs where cudaMalloc is not allowed or not wanted -- inside a
+// region whose memory was planned ahead of time by an inference runtime, a
+// plugin whose host framework owns every allocation, or a real-time loop where
+// an allocator call could stall or fail. gdn_prefill needs a workspace (the
+// package ring the preparation and chain CTAs exchange data through), so for
+// those callers this file keeps one statically sized scratch array in device
+// memory and gdn_prefill_noalloc runs the same kernel on it.
+//
+// The array lives as long as the library is loaded, on every device that
+// loads it. Its device address is looked up once per device (first call with
+// that device current) with cudaGetSymbolAddress; host code must never use
+// the array's name as a device pointer. Every call shares the array: the
+// parts that must start at zero are cleared by each call on its stream, and
+// two calls whose kernels overlap on the GPU (different streams, or different
+// host threads) race on it and must be serialised by the caller.
+// ============================================================================
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 64ull << 20;   // 64 MiB
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+gdn_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "gdn_prefill_noalloc: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices)
+    return fail(GDN_ERR_UNSUPPORTED, "gdn_prefill_noalloc: device %d beyond %d", dev, kMaxDevices);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess || !ptr)
+      return fail(GDN_ERR_CUDA, "gdn_prefill_noalloc: cudaGetSymbolAddress failed: %s",
+                  cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return GDN_OK;
+}
+
+}  // namespace
+
+extern "C" gdn_status gdn_prefill_noalloc(const void* q, const void* k, const void* v, const float* g,
+                                          const float* beta, const float* state_in,
+                                          const int32_t* cu_seqlens, int n_seqs, int64_t total_T, int Hqk,
+                                          int Hv, int dk, int dv, float scale, int chunk, gdn_dtype dtype,
+                                          void* o, float* state_out, void* stream) {
+  if (dtype != GDN_BF16 || dk != 128 || dv != 128 || (chunk != 0 && chunk != 64))
+    return fail(GDN_ERR_UNSUPPORTED,
+                "gdn_prefill_noalloc: only bf16 with dk = dv = 128 and chunk 64 (the tensor-core kernel)");
+  if (n_seqs > 0 && Hv > 0) {
+    const size_t need = gdn::pc::Workspace::bytes((long)n_seqs * Hv);
+    if (need > kNoAllocScratchBytes)
+      return fail(GDN_ERR_UNSUPPORTED,
+                  "gdn_prefill_noalloc: %d sequences x %d heads need %zu bytes of scratch, more than the %zu "
+                  "bytes built into the library; use gdn_prefill with a workspace",
+                  n_seqs, Hv, need, kNoAllocScratchBytes);
+  }
+  void* scratch = nullptr;
+  if (gdn_status s = noalloc_scratch(&scratch)) return s;
+  return gdn_prefill(q, k, v, g, beta, state_in, cu_seqlens, n_seqs, total_T, Hqk, Hv, dk, dv, scale, chunk,
+                     dtype, o, state_out, scratch, kNoAllocScratchBytes, stream);
+}

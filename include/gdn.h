@@ -110,6 +110,37 @@ gdn_status gdn_prefill(const void *q, const void *k, const void *v,
                        void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Allocation-free variant of gdn_prefill for callers that cannot provide
+ * device scratch memory of their own: code running inside memory that an
+ * inference runtime planned ahead of time, plugins whose host framework owns
+ * every allocation, or real-time loops that must not call an allocator. The
+ * Herbert pages have no counterpart to it; it exists for integration only.
+ *
+ * It runs the same tensor-core prefill as gdn_prefill, with the workspace
+ * taken from a scratch array compiled into the library (64 MiB of device
+ * memory held on every device that loads the library, until the process
+ * exits). It calls no allocator. Arguments are those of gdn_prefill without
+ * the workspace; the caller still passes every input and output.
+ *
+ *   Supported: GDN_BF16, dk = dv = 128, chunk 0 or 64. Problems whose workspace
+ *   (gdn_prefill_workspace_bytes) exceeds 64 MiB -- more than about 320
+ *   sequence-heads -- return GDN_ERR_UNSUPPORTED with a message.
+ *   The first call on each device looks up the array's device address with
+ *   cudaGetSymbolAddress (with that device current); make that first call
+ *   before capturing the stream into a CUDA graph.
+ *   All calls share the one array and each call clears the part that must
+ *   start at zero on its stream: calls whose kernels can overlap on the GPU
+ *   (different streams or host threads) race and must be serialised by the
+ *   caller.
+ */
+gdn_status gdn_prefill_noalloc(const void *q, const void *k, const void *v,
+                               const float *g, const float *beta,
+                               const float *state_in, const int32_t *cu_seqlens,
+                               int n_seqs, int64_t total_T, int Hqk, int Hv, int dk, int dv,
+                               float scale, int chunk, gdn_dtype dtype,
+                               void *o, float *state_out, void *stream);
+
+/*
  * One decode step for B independent sequences, one token each; the fused
  * step of "One level down: #004 the same compiler on Apple's chips",
  * section "Decode": L2-normalise q and k, decay, rank-1 delta update and
