@@ -222,7 +222,9 @@ gdn_status launch_prefill_pc(const void* q, const void* k, const void* v, const 
   }
   const int slices = 128 / dvp;
   long nc = (long)(sms * 0.45);
+  if (const char* env = getenv("GDN_PC_NC")) nc = std::max(1, std::min(atoi(env), sms - 1));
   nc = std::min(nc, chains * slices);
+  nc = std::min(nc, (long)gdn::pc::kMaxPositions * slices);
   nc -= nc % slices;
   if (nc < slices) nc = slices;
   const long rounds = (chains * slices + nc - 1) / nc;
@@ -232,7 +234,7 @@ gdn_status launch_prefill_pc(const void* q, const void* k, const void* v, const 
   if (!make_map(&qm, q, 128, Hqk, (int)total_T, 64) || !make_map(&km, k, 128, Hqk, (int)total_T, 64) ||
       !make_map(&vm, v, 128, Hv, (int)total_T, dvp))
     return fail(GDN_ERR_CUDA, "gdn_prefill: cuTensorMapEncodeTiled unavailable or failed");
-  cudaError_t e = cudaMemsetAsync(ws, 0, gdn::pc::Workspace::zeroed_bytes(chains), st);
+  cudaError_t e = cudaMemsetAsync(ws, 0, gdn::pc::Workspace::zeroed_bytes(nc / slices), st);
   if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "gdn_prefill: %s", cudaGetErrorString(e));
   gdn::pc::Params prm;
   prm.g = g;
@@ -275,7 +277,7 @@ const char* gdn_last_error(void) { return t_last_error.c_str(); }
 
 size_t gdn_prefill_workspace_bytes(int n_seqs, int Hv, int dk, int dv, gdn_dtype dtype) {
   if (n_seqs <= 0 || Hv <= 0 || !uses_pc_prefill(dtype, dk, dv)) return 0;
-  return gdn::pc::Workspace::bytes((long)n_seqs * Hv);
+  return gdn::pc::Workspace::bytes(std::min((long)n_seqs * Hv, (long)gdn::pc::kMaxPositions));
 }
 
 gdn_status gdn_prefill(const void* q, const void* k, const void* v, const float* g,
@@ -391,7 +393,10 @@ gdn_status gdn_device_error(void* stream) {
 // ============================================================================
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = 64ull << 20;   // 64 MiB
+// The largest workspace gdn_prefill can ask for (the ring of kMaxPositions
+// positions), rounded up to whole MiB: every problem gdn_prefill runs fits.
+constexpr size_t kNoAllocScratchBytes =
+    (gdn::pc::Workspace::bytes(gdn::pc::kMaxPositions) + (size_t(1) << 20) - 1) & ~((size_t(1) << 20) - 1);
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
@@ -428,7 +433,7 @@ extern "C" gdn_status gdn_prefill_noalloc(const void* q, const void* k, const vo
     return fail(GDN_ERR_UNSUPPORTED,
                 "gdn_prefill_noalloc: only bf16 with dk = dv = 128 and chunk 64 (the tensor-core kernel)");
   if (n_seqs > 0 && Hv > 0) {
-    const size_t need = gdn::pc::Workspace::bytes((long)n_seqs * Hv);
+    const size_t need = gdn_prefill_workspace_bytes(n_seqs, Hv, dk, dv, dtype);
     if (need > kNoAllocScratchBytes)
       return fail(GDN_ERR_UNSUPPORTED,
                   "gdn_prefill_noalloc: %d sequences x %d heads need %zu bytes of scratch, more than the %zu "

@@ -56,10 +56,16 @@ def test_noalloc_prefill_matches_workspace_prefill_twice(call):
         assert (s - s_ref).abs().max().item() <= 1e-2
 
 
-def test_noalloc_rejects_problems_beyond_its_scratch():
+def test_noalloc_scratch_covers_every_workspace_and_rejects_other_kernels():
     lib = gdn.lib()
-    P = 0x10000   # never dereferenced: the size check fails first
-    status = lib.gdn_prefill_noalloc(P, P, P, P, P, None, P, 10000, 10000, 16, 32, 128, 128,
-                                     ctypes.c_float(0.0), 0, gdn.GDN_BF16, P, P, None)
+    # the workspace is bounded however many sequences there are, so the
+    # built-in scratch (sized for the largest) serves every problem
+    assert lib.gdn_prefill_workspace_bytes(10000, 32, 128, 128, gdn.GDN_BF16) == \
+        lib.gdn_prefill_workspace_bytes(100000, 64, 128, 128, gdn.GDN_BF16)
+    P = 0x10000   # never dereferenced: argument checks fail first
+    status = lib.gdn_prefill_noalloc(P, P, P, P, P, None, P, 1, 64, 2, 2, 128, 128,
+                                     ctypes.c_float(0.0), 0, gdn.GDN_F32, P, P, None)
     assert status == gdn.GDN_ERR_UNSUPPORTED
-    assert "scratch" in lib.gdn_last_error().decode()
+    status = lib.gdn_prefill_noalloc(P, P, P, P, P, None, P, 1, 64, 2, 2, 128, 128,
+                                     ctypes.c_float(0.0), 32, gdn.GDN_BF16, P, P, None)
+    assert status == gdn.GDN_ERR_UNSUPPORTED
