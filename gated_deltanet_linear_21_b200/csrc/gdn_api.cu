@@ -1,5 +1,6 @@
 // C ABI of libgdn.so: argument checks, kernel selection and launches.
 // Declared and documented in include/gdn.h.
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -190,7 +191,7 @@ bool uses_pc_prefill(gdn_dtype dtype, int dk, int dv) {
 }
 
 template <int DVP>
-gdn_status launch_pc(const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm,
+gdn_status launch_pc(const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& om,
                      const gdn::pc::Params& prm, int grid, cudaStream_t st) {
   auto kern = gdn::pc::prefill_pc_kernel<DVP>;
   if (gdn_status s = allow_smem(kern, "gdn_prefill")) return s;
@@ -204,9 +205,41 @@ gdn_status launch_pc(const CUtensorMap& qm, const CUtensorMap& km, const CUtenso
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, qm, km, vm, prm);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, qm, km, vm, om, prm);
   if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "gdn_prefill: launch failed: %s", cudaGetErrorString(e));
   return launch_status("gdn_prefill");
+}
+
+// Chooses the state slice width DVP and the number of chain CTAs. The kernel
+// runs min(NC, slice-chains) state chains at a time, in rounds, and prepares
+// packages on the remaining CTAs; its time is about the larger of the two
+// sides. Per-chunk costs (SM cycles) measured on B200: a chain step of one
+// slice and the preparation of one (head, chunk) item.
+struct PcPlan {
+  int dvp;
+  long nc;
+};
+PcPlan plan_pc(long chains, int64_t total_T, int n_seqs, int sms) {
+  const double kChainStep[3] = {2300.0, 2800.0, 3600.0};   // DVP 32, 64, 128
+  const double kPrepItem = 12700.0;
+  const double chunks = std::max(1.0, std::ceil((double)total_T / std::max(1, n_seqs) / 64.0));
+  PcPlan best = {128, 1};
+  double best_t = 1e300;
+  for (int t = 0; t < 3; ++t) {
+    const int dvp = 32 << t, slices = 128 / dvp;
+    const long nc_max = std::min({chains * slices, (long)gdn::pc::kMaxPositions * slices, (long)sms - 8});
+    for (long nc = slices; nc <= nc_max; nc += slices) {
+      const double rounds = std::ceil((double)(chains * slices) / nc);
+      const double chain_t = rounds * chunks * kChainStep[t];
+      const double prep_t = chains * chunks * kPrepItem / (double)(sms - nc);
+      const double tt = std::max(chain_t, prep_t);
+      if (tt < best_t * 0.999) {
+        best_t = tt;
+        best = {dvp, nc};
+      }
+    }
+  }
+  return best;
 }
 
 gdn_status launch_prefill_pc(const void* q, const void* k, const void* v, const float* g, const float* beta,
@@ -214,14 +247,14 @@ gdn_status launch_prefill_pc(const void* q, const void* k, const void* v, const 
                              int Hv, float scale, void* o, float* state_out, void* ws, cudaStream_t st) {
   const long chains = (long)n_seqs * Hv;
   const int sms = sm_count();
-  if (sms < 4) return fail(GDN_ERR_CUDA, "gdn_prefill: cannot query the multiprocessor count");
-  int dvp = chains * 4 <= (long)(sms * 0.45) ? 32 : 64;
+  if (sms < 16) return fail(GDN_ERR_CUDA, "gdn_prefill: cannot query the multiprocessor count");
+  PcPlan plan = plan_pc(chains, total_T, n_seqs, sms);
   if (const char* env = getenv("GDN_TC_SLICE")) {
     const int v2 = atoi(env);
-    if (v2 == 32 || v2 == 64) dvp = v2;
+    if (v2 == 32 || v2 == 64 || v2 == 128) plan.dvp = v2;
   }
-  const int slices = 128 / dvp;
-  long nc = (long)(sms * 0.45);
+  const int dvp = plan.dvp, slices = 128 / dvp;
+  long nc = plan.nc;
   if (const char* env = getenv("GDN_PC_NC")) nc = std::max(1, std::min(atoi(env), sms - 1));
   nc = std::min(nc, chains * slices);
   nc = std::min(nc, (long)gdn::pc::kMaxPositions * slices);
@@ -230,9 +263,10 @@ gdn_status launch_prefill_pc(const void* q, const void* k, const void* v, const 
   const long rounds = (chains * slices + nc - 1) / nc;
   if (rounds > gdn::pc::kMaxRounds)
     return fail(GDN_ERR_UNSUPPORTED, "gdn_prefill: %ld sequence-heads is more than this kernel schedules", chains);
-  CUtensorMap qm, km, vm;
+  CUtensorMap qm, km, vm, om;
   if (!make_map(&qm, q, 128, Hqk, (int)total_T, 64) || !make_map(&km, k, 128, Hqk, (int)total_T, 64) ||
-      !make_map(&vm, v, 128, Hv, (int)total_T, dvp))
+      !make_map(&vm, v, 128, Hv, (int)total_T, std::min(dvp, 64)) ||
+      !make_map(&om, o, 128, Hv, (int)total_T, std::min(dvp, 64)))
     return fail(GDN_ERR_CUDA, "gdn_prefill: cuTensorMapEncodeTiled unavailable or failed");
   cudaError_t e = cudaMemsetAsync(ws, 0, gdn::pc::Workspace::zeroed_bytes(nc / slices), st);
   if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "gdn_prefill: %s", cudaGetErrorString(e));
@@ -250,8 +284,9 @@ gdn_status launch_prefill_pc(const void* q, const void* k, const void* v, const 
   prm.total_T = (int)total_T;
   prm.scale = scale;
   prm.n_chain_ctas = (int)nc;
-  if (dvp == 32) return launch_pc<32>(qm, km, vm, prm, sms, st);
-  return launch_pc<64>(qm, km, vm, prm, sms, st);
+  if (dvp == 32) return launch_pc<32>(qm, km, vm, om, prm, sms, st);
+  if (dvp == 64) return launch_pc<64>(qm, km, vm, om, prm, sms, st);
+  return launch_pc<128>(qm, km, vm, om, prm, sms, st);
 }
 
 gdn_status launch_prefill_tc(const void* q, const void* k, const void* v, const float* g, const float* beta,

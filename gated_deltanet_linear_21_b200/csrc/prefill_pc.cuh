@@ -124,6 +124,11 @@ constexpr uint32_t kColDS = 128;   // chain: dS^T           M=128, N=DVP
 
 template <int DVP>
 struct Smem {
+  // A slice of DVP state rows is stored as blocks of kBlk columns, each an
+  // MN-major tile with rows of kRB bytes and the matching swizzle.
+  static constexpr int kBlk = DVP < 64 ? DVP : 64;
+  static constexpr int kBlocks = DVP / kBlk;
+  static constexpr uint32_t kRB = kBlk * 2;
   static constexpr uint32_t kR = DVP * 2;
   // chain role: two input buffers {package image, k tile, v slice}
   static constexpr uint32_t kIn = 0;
@@ -144,24 +149,30 @@ struct Smem {
   static constexpr uint32_t kTw = kPm + 8192;                 // -T_w
   static constexpr uint32_t kTu = kTw + 8192;                 // T_u
   static constexpr uint32_t kWm = kTu + 8192;                 // -W [64][128], two halves 8 KB apart
-  static constexpr uint32_t kAd = kWm + 16384;                // diagonal blocks of A, fp32 [4][16][16]
+  static constexpr uint32_t kA1b = kWm + 16384;               // rho Q - P W [64][128], two halves 8 KB apart
+  static constexpr uint32_t kA2b = kA1b + 16384;              // P T_u [64][64]
+  static constexpr uint32_t kPv = kA2b + 8192;                // package vectors: us[64], gamma_L, tokens
+  static constexpr uint32_t kAd = kPv + 1024;                 // diagonal blocks of A, fp32 [4][16][16]
   static constexpr uint32_t kVec = kAd + 4096;                // 8 vectors of 64 fp32
   static constexpr uint32_t kQueue = kVec + 8 * 256;          // 2 items handed over by the control warp:
   static constexpr uint32_t kQueueBytes = 640;                //   {valid, s, q, len}, g[64] @64, beta[64] @320
-  static constexpr uint32_t kPrepEnd = kQueue + 2 * kQueueBytes;
-  // common
-  static constexpr uint32_t kCommon = ((kChainEnd > kPrepEnd ? kChainEnd : kPrepEnd) + 1023) & ~1023u;
-  static constexpr uint32_t kRounds = kCommon;                // round_start[kMaxRounds + 1]
+  static constexpr uint32_t kRounds = kQueue + 2 * kQueueBytes;      // round_start[kMaxRounds + 1]
   static constexpr uint32_t kRBase = kRounds + 4 * (kMaxRounds + 1);   // base_r [kMaxRounds + 1]
-  static constexpr uint32_t kBar = kRBase + 4 * (kMaxRounds + 1) + 12;
-  static constexpr uint32_t kBarA = (kBar + 7) & ~7u;         // full[2], free[2], mma
+  static constexpr uint32_t kPrepEnd = kRBase + 4 * (kMaxRounds + 1);
+  // common
+  static constexpr uint32_t kCommon = ((kChainEnd > kPrepEnd ? kChainEnd : kPrepEnd) + 7) & ~7u;
+  static constexpr uint32_t kBarA = kCommon;                  // full[2], free[2], mma
   static constexpr uint32_t kMisc = kBarA + 5 * 8;            // tmem slot, scan[4]
   static constexpr uint32_t kTotal = kMisc + 64;
   static constexpr uint32_t kAlloc = kTotal + 1024;
   static_assert(kAlloc <= 227 * 1024, "shared memory budget");
   static_assert((kInBytes % 1024) == 0 && (kInK % 1024) == 0 && (kInV % 1024) == 0 && (kUsb % 1024) == 0 &&
-                    (kSb % 1024) == 0 && (kWm % 1024) == 0,
+                    (kSb % 1024) == 0 && (kWm % 1024) == 0 && (kA1b % 1024) == 0 && (kA2b % 1024) == 0,
                 "tile alignment");
+  // byte offset of element (row, col) of a slice tile with `rows` rows
+  __device__ static __forceinline__ uint32_t tile_off(int row, int col, int rows) {
+    return (uint32_t)(col / kBlk) * (uint32_t)rows * kRB + sm100::mn_off<kRB>(row, col % kBlk);
+  }
 };
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
@@ -203,13 +214,15 @@ struct Params {
 template <int DVP>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
-                  const __grid_constant__ CUtensorMap vmap, const Params p) {
+                  const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap omap,
+                  const Params p) {
   using L = Smem<DVP>;
   using namespace sm100;
-  static_assert(DVP == 32 || DVP == 64, "slice width");
+  static_assert(DVP == 32 || DVP == 64 || DVP == 128, "slice width");
   constexpr int kSlices = kD / DVP;
   constexpr int kHalf = DVP / 2;
-  constexpr uint32_t kR = L::kR;
+  constexpr uint32_t kR = L::kR, kRB = L::kRB;
+  constexpr int kPart = kHalf;   // epilogue columns per TMEM load
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(sm);
@@ -253,7 +266,10 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     fence_mbar_init();
     prefetch_tensormap(&qmap);
     prefetch_tensormap(&kmap);
-    if (is_chain) prefetch_tensormap(&vmap);
+    if (is_chain) {
+      prefetch_tensormap(&vmap);
+      prefetch_tensormap(&omap);
+    }
   }
   if (warp == 0) {
     tmem_alloc(&misc[0], kTmemCols);
@@ -301,6 +317,19 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       uint32_t* rdy = ready + q * kRing;
       uint32_t* cns = consumed + q * kRing;
       const uint8_t* ring = pkgs + (size_t)q * kRing * kPkgStride;
+      // Copies whose ring slot is not handed back yet, per input buffer (lane 0's
+      // copy of these is the one that counts). A slot goes back as soon as its copy
+      // has landed; the warp never waits for that while it could issue a copy.
+      bool pend[2] = {false, false};
+      int pend_slot[2] = {0, 0};
+      long pend_gc[2] = {0, 0};
+      auto release0 = [&](int bb, bool block) {
+        if (!pend[bb]) return;
+        const uint32_t par = (uint32_t)(pend_gc[bb] >> 1) & 1u;
+        if (block ? !mbar_wait(&bar_full[bb], par) : !mbar_test_wait(&bar_full[bb], par)) return;
+        red_add_release_gpu(&cns[pend_slot[bb]], 1u);
+        pend[bb] = false;
+      };
       long gc = 0;
       int base = 0;
       for (long sc = blockIdx.x; sc < n_slice_chains && !abort; sc += NC) {
@@ -319,9 +348,22 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           const int b = (int)(gc & 1);
           const int s = base + c, slot = s % kRing;
           bool ok = true;
-          if (lane == 0) ok = wait_flag_geq(&rdy[slot], (uint32_t)(s / kRing + 1));
+          if (lane == 0) {   // wait for the package, handing back the other buffer's slot meanwhile
+            const uint32_t want = (uint32_t)(s / kRing + 1);
+            const long long t0 = clock64();
+            while (ld_acquire_gpu(&rdy[slot]) < want) {
+              release0(b ^ 1, false);
+              if (clock64() - t0 > 4000000000ll) {
+                flag_error(kErrTimeout);
+                ok = false;
+                break;
+              }
+              __nanosleep(64);
+            }
+          }
           if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) { abort = true; break; }
           if (gc >= 2 && !mbar_wait(&bar_free[b], (uint32_t)((gc - 2) >> 1) & 1u)) { abort = true; break; }
+          if (lane == 0) release0(b, true);   // (landed: its chunk has been computed)
           fence_async_global();
           uint8_t* dst = sm + L::kIn + b * L::kInBytes;
           const int c0 = t_begin + c * kC;
@@ -329,14 +371,21 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           bulk_load_warp(dst, ring + (size_t)slot * kPkgStride, kPkgCopy, &bar_full[b]);
           tma_load_3d_warp(dst + L::kInK, &kmap, &bar_full[b], 0, hq, c0);
           tma_load_3d_warp(dst + L::kInK + 8192, &kmap, &bar_full[b], 64, hq, c0);
-          tma_load_3d_warp(dst + L::kInV, &vmap, &bar_full[b], i0, h, c0);
-          if (!mbar_wait(&bar_full[b], (uint32_t)(gc >> 1) & 1u)) { abort = true; break; }
-          if (lane == 0) red_add_release_gpu(&cns[slot], 1u);
+#pragma unroll
+          for (int vb = 0; vb < L::kBlocks; ++vb)
+            tma_load_3d_warp(dst + L::kInV + vb * 64 * L::kRB, &vmap, &bar_full[b], i0 + vb * L::kBlk, h, c0);
+          pend[b] = true;
+          pend_slot[b] = slot;
+          pend_gc[b] = gc;
         }
         if (abort) break;
         if (lane == 0)   // numbers this chain leaves unused count as read
           for (int c = nch; c < maxc; ++c) red_add_release_gpu(&cns[(base + c) % kRing], 1u);
         base += maxc;
+      }
+      if (lane == 0) {   // hand back what is still out (bounded waits)
+        release0(0, true);
+        release0(1, true);
       }
     } else {
       // ---- compute warps ----
@@ -349,7 +398,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         const uint32_t in = sbase + L::kIn + b * L::kInBytes;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16_warp(tmem + kColY, desc_kmajor(in + kPkgA2, kk, 0), desc_mnmajor(in + L::kInV, kk, kR, 64 * kR),
+          mma_bf16_warp(tmem + kColY, desc_kmajor(in + kPkgA2, kk, 0), desc_mnmajor(in + L::kInV, kk, kRB, 64 * kRB),
                         kIdY, kk > 0);
       };
       long gc = 0;
@@ -368,7 +417,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         auto store_state = [&]() {
 #pragma unroll
           for (int c8 = 0; c8 < kHalf / 8; ++c8)
-            st_shared_v4(sSb + mn_off<kR>(r128, ch * kHalf + 8 * c8), pack8_bf16(Sreg + 8 * c8));
+            st_shared_v4(sSb + L::tile_off(r128, ch * kHalf + 8 * c8, 128), pack8_bf16(Sreg + 8 * c8));
         };
         store_state();
         publish();
@@ -386,38 +435,54 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
               if (!early) issue_a2v(b);
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk)
-                mma_bf16_warp(tmem + kColY, desc_kmajor(in + kPkgA1, kk, 16384), desc_mnmajor(sSb, kk, kR, 128 * kR),
+                mma_bf16_warp(tmem + kColY, desc_kmajor(in + kPkgA1, kk, 16384), desc_mnmajor(sSb, kk, kRB, 128 * kRB),
                               kIdY, 1u);
             }
             mma_commit_warp(bar_mma);
           }
           if (!wait_mma(full_ok)) { abort = true; break; }
+          // O of a whole chunk goes out by TMA from the v tile's place (v is consumed);
+          // the rows of a sequence's last, partial chunk are stored one by one
+          const bool o_tma = len == kC;
           {
-            float yv[kHalf];
-            tmem_ld<kHalf>(tmem + tlane + kColY + ch * kHalf, yv);
-            if (qd < 2) {   // U_s = diag(us) U -> shared memory (bf16) for dS
-              const float us = reinterpret_cast<const float*>(in_g + kPkgUs)[r128];
+            const float us = qd < 2 ? reinterpret_cast<const float*>(in_g + kPkgUs)[r128] : 0.f;
+            __nv_bfloat16* orow = p.o + ((size_t)(t_begin + c * kC + (r128 & 63)) * Hv + h) * kD + i0 + ch * kHalf;
 #pragma unroll
-              for (int q2 = 0; q2 < kHalf; ++q2) yv[q2] *= us;
+            for (int pp = 0; pp < kHalf / kPart; ++pp) {
+              float yv[kPart];
+              tmem_ld<kPart>(tmem + tlane + kColY + ch * kHalf + pp * kPart, yv);
+              if (qd < 2) {   // U_s = diag(us) U -> shared memory (bf16) for dS
 #pragma unroll
-              for (int c8 = 0; c8 < kHalf / 8; ++c8)
-                st_shared_v4(sUsb + mn_off<kR>(r128, ch * kHalf + 8 * c8), pack8_bf16(yv + 8 * c8));
-            } else if (r128 - 64 < len) {   // O rows -> global
-              const int r = r128 - 64;
-              __nv_bfloat16* orow = p.o + ((size_t)(t_begin + c * kC + r) * Hv + h) * kD + i0 + ch * kHalf;
+                for (int q2 = 0; q2 < kPart; ++q2) yv[q2] *= us;
 #pragma unroll
-              for (int c8 = 0; c8 < kHalf / 8; ++c8)
-                *reinterpret_cast<uint4*>(orow + 8 * c8) = pack8_bf16(yv + 8 * c8);
+                for (int c8 = 0; c8 < kPart / 8; ++c8)
+                  st_shared_v4(sUsb + L::tile_off(r128, ch * kHalf + pp * kPart + 8 * c8, 64), pack8_bf16(yv + 8 * c8));
+              } else if (o_tma) {
+#pragma unroll
+                for (int c8 = 0; c8 < kPart / 8; ++c8)
+                  st_shared_v4(in + L::kInV + L::tile_off(r128 - 64, ch * kHalf + pp * kPart + 8 * c8, 64),
+                               pack8_bf16(yv + 8 * c8));
+              } else if (r128 - 64 < len) {
+#pragma unroll
+                for (int c8 = 0; c8 < kPart / 8; ++c8)
+                  *reinterpret_cast<uint4*>(orow + pp * kPart + 8 * c8) = pack8_bf16(yv + 8 * c8);
+              }
             }
           }
           publish();
+          if (tid == 0 && o_tma) {
+#pragma unroll
+            for (int vb = 0; vb < L::kBlocks; ++vb)
+              tma_store_3d(&omap, in_g + L::kInV + vb * 64 * kRB, i0 + vb * L::kBlk, h, t_begin + c * kC);
+            bulk_commit_group();
+          }
 
           // ---- dS^T = K_raw^T U_s ; then, if the next chunk is in, its A2 V ----
           if (warp == 0) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               mma_bf16_warp(tmem + kColDS, desc_mnmajor(in + L::kInK, kk, 128, 8192),
-                            desc_mnmajor(sUsb, kk, kR, 64 * kR), kIdDS, kk > 0);
+                            desc_mnmajor(sUsb, kk, kRB, 64 * kRB), kIdDS, kk > 0);
             mma_commit_warp(bar_mma);
             early = false;
             if (c + 1 < nch) {
@@ -430,15 +495,21 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           }
           if (!wait_mma()) { abort = true; break; }
           {
-            float ds[kHalf];
-            tmem_ld<kHalf>(tmem + tlane + kColDS + ch * kHalf, ds);
             const float gL = *reinterpret_cast<const float*>(in_g + kPkgGL);
 #pragma unroll
-            for (int q2 = 0; q2 < kHalf; ++q2) Sreg[q2] = fmaf(gL, Sreg[q2], ds[q2]);
+            for (int pp = 0; pp < kHalf / kPart; ++pp) {
+              float ds[kPart];
+              tmem_ld<kPart>(tmem + tlane + kColDS + ch * kHalf + pp * kPart, ds);
+#pragma unroll
+              for (int q2 = 0; q2 < kPart; ++q2) Sreg[pp * kPart + q2] = fmaf(gL, Sreg[pp * kPart + q2], ds[q2]);
+            }
             store_state();
           }
           publish();
-          if (tid == 0) mbar_arrive(&bar_free[b]);
+          if (tid == 0) {
+            bulk_wait_read_all();   // the O tile has left the buffer
+            mbar_arrive(&bar_free[b]);
+          }
         }
         if (abort) break;
 #pragma unroll
@@ -594,9 +665,22 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       float* Ad = reinterpret_cast<float*>(sm + L::kAd);
       float* scan = reinterpret_cast<float*>(&misc[2]);
 
+      // Thread 0: once the bulk copies of the previous package are complete, order
+      // them before the control warp's release and hand the item back.
+      int out_pending = -1;
+      auto finish_out = [&]() {
+        if (out_pending < 0) return;
+        bulk_wait_all();
+        fence_async_global();
+        mbar_arrive(&bar_free[out_pending]);
+        out_pending = -1;
+      };
       for (int it = 0; !abort; ++it) {
         const int b = it & 1;
         const uint32_t* qe = reinterpret_cast<const uint32_t*>(sm + L::kQueue + b * L::kQueueBytes);
+        // The previous package is published during this item's first stage, unless
+        // this item is not here yet: its ring slot may wait for that package.
+        if (tid == 0 && out_pending >= 0 && !mbar_test_wait(&bar_full[b], (uint32_t)(it >> 1) & 1u)) finish_out();
         {
           const bool w = mbar_wait(&bar_full[b], (uint32_t)(it >> 1) & 1u);
           if (!cbar_and(w)) { abort = true; break; }
@@ -612,39 +696,39 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           for (int kk = 0; kk < 8; ++kk)
             mma_bf16_warp(tmem + kColG, desc_kmajor(sKQ, kk, 16384), desc_kmajor(sKQ, kk, 16384), kIdG, kk > 0);
           mma_commit_warp(bar_mma);
+          if (lane == 0) finish_out();   // (before this item's vectors reuse the staging)
         }
-        if (tid < 64) {   // inclusive scan of g within each warp; the halves are joined below
-          float gv = reinterpret_cast<const float*>(qe + 16)[tid];
+        if (warp == 2 || warp == 3) {   // inclusive scan of g within each warp; the halves are joined below
+          const int t = tid - 64, w2 = warp - 2;
+          float gv = reinterpret_cast<const float*>(qe + 16)[t];
           const unsigned nonpos = __ballot_sync(0xffffffffu, gv <= 0.f);
 #pragma unroll
           for (int off = 1; off < 32; off <<= 1) {
             const float up = __shfl_up_sync(0xffffffffu, gv, off);
             if (lane >= off) gv += up;
           }
-          if (lane == 31) scan[warp] = gv;
-          if (lane == 0) scan[2 + warp] = nonpos == 0xffffffffu ? 1.f : 0.f;
-          vB[tid] = reinterpret_cast<const float*>(qe + 80)[tid];
-          vG[tid] = gv;
-        }
-        {
-          const int row = tid >> 1, half = tid & 1;   // rows 0-63: k, rows 64-127: q
-          float ss = 0.f;
+          if (lane == 31) scan[w2] = gv;
+          if (lane == 0) scan[2 + w2] = nonpos == 0xffffffffu ? 1.f : 0.f;
+          vB[t] = reinterpret_cast<const float*>(qe + 80)[t];
+          vG[t] = gv;
+        } else if (warp >= 4) {   // norms, one row each: rows 0-63 k, rows 64-127 q
+          const int row = tid - 128;
+          float ss0 = 0.f, ss1 = 0.f;
 #pragma unroll
-          for (int c8 = 0; c8 < 8; ++c8) {
-            const uint4 raw = ld_shared_v4(sKQ + sw128_off(row, 64 * half + 8 * c8, 16384));
+          for (int c8 = 0; c8 < 16; ++c8) {
+            const uint4 raw = ld_shared_v4(sKQ + sw128_off(row, 8 * c8, 16384));
             const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const float2 f = __bfloat1622float2(p2[e]);
-              ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+              if (e & 1) ss1 = fmaf(f.x, f.x, fmaf(f.y, f.y, ss1));
+              else ss0 = fmaf(f.x, f.x, fmaf(f.y, f.y, ss0));
             }
           }
-          ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-          if (half == 0) {
-            const int rr = row & 63;
-            if (row < 64) vRk[rr] = rr < len ? 1.0f / sqrtf(ss + kNormEps) : 0.f;
-            else vRq[rr] = rr < len ? p.scale / sqrtf(ss + kNormEps) : 0.f;
-          }
+          const float ss = ss0 + ss1;
+          const int rr = row & 63;
+          if (row < 64) vRk[rr] = rr < len ? 1.0f / sqrtf(ss + kNormEps) : 0.f;
+          else vRq[rr] = rr < len ? p.scale / sqrtf(ss + kNormEps) : 0.f;
         }
         cbar();
 
@@ -662,10 +746,10 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           vCk[tid] = fast ? expf(gm - Gr) * rk : rk;
           vCw[tid] = -vB[tid] * eg * rk;
           vRho[tid] = eg * vRq[tid];
-          reinterpret_cast<float*>(pkg + kPkgUs)[tid] = expf(GL - Gr) * rk;
+          reinterpret_cast<float*>(sm + L::kPv)[tid] = expf(GL - Gr) * rk;
           if (tid == 0) {
-            reinterpret_cast<float*>(pkg + kPkgGL)[0] = expf(GL);
-            reinterpret_cast<int*>(pkg + kPkgGL)[1] = len;
+            reinterpret_cast<float*>(sm + L::kPv + 256)[0] = expf(GL);
+            reinterpret_cast<int*>(sm + L::kPv + 256)[1] = len;
           }
         }
         if (!wait_mma()) { abort = true; break; }   // (its barrier also publishes the vectors)
@@ -840,9 +924,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
                 tw[e] = t * vCw[sidx];
               }
               const uint32_t off = sw128_off(r64, 32 * ch + 8 * c8, 0);
-              const uint4 u4 = pack8_bf16(tu);
-              st_shared_v4(sbase + L::kTu + off, u4);
-              st_global_v4(pkg + kPkgA2 + off, u4);
+              st_shared_v4(sbase + L::kTu + off, pack8_bf16(tu));
               st_shared_v4(sbase + L::kTw + off, pack8_bf16(tw));
             }
           }
@@ -858,17 +940,14 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           mma_commit_warp(bar_mma);
         }
         if (!wait_mma()) { abort = true; break; }
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          float w[32];
-          tmem_ld32(tmem + tlane + kColW + 64 * ch + 32 * hh, w);
+        {
+          float w[64];
+          tmem_ld64(tmem + tlane + kColW + 64 * ch, w);
           if (lo16) {
 #pragma unroll
-            for (int c8 = 0; c8 < 4; ++c8) {
-              const int d = 64 * ch + 32 * hh + 8 * c8;
-              const uint4 w4 = pack8_bf16(w + 8 * c8);
-              st_shared_v4(sbase + L::kWm + sw128_off(r64, d, 8192), w4);
-              st_global_v4(pkg + kPkgA1 + sw128_off(r64, d, 16384), w4);
+            for (int c8 = 0; c8 < 8; ++c8) {
+              const int d = 64 * ch + 8 * c8;
+              st_shared_v4(sbase + L::kWm + sw128_off(r64, d, 8192), pack8_bf16(w + 8 * c8));
             }
           }
         }
@@ -889,16 +968,14 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         if (!wait_mma()) { abort = true; break; }
         {
           const float rho = vRho[r64];
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            float pw[32];
-            tmem_ld32(tmem + tlane + kColPW + 64 * ch + 32 * hh, pw);
+          {
+            float pw[64];
+            tmem_ld64(tmem + tlane + kColPW + 64 * ch, pw);
             if (lo16) {
 #pragma unroll
-              for (int c8 = 0; c8 < 4; ++c8) {
-                const int d = 64 * ch + 32 * hh + 8 * c8;
-                const uint32_t off = sw128_off(64 + r64, d, 16384);
-                const uint4 qv = ld_shared_v4(sKQ + off);
+              for (int c8 = 0; c8 < 8; ++c8) {
+                const int d = 64 * ch + 8 * c8;
+                const uint4 qv = ld_shared_v4(sKQ + sw128_off(64 + r64, d, 16384));
                 const __nv_bfloat162* q2v = reinterpret_cast<const __nv_bfloat162*>(&qv);
                 float a[8];
 #pragma unroll
@@ -907,7 +984,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
                   a[2 * e] = fmaf(rho, qf.x, pw[8 * c8 + 2 * e]);
                   a[2 * e + 1] = fmaf(rho, qf.y, pw[8 * c8 + 2 * e + 1]);
                 }
-                st_global_v4(pkg + kPkgA1 + off, pack8_bf16(a));
+                st_shared_v4(sbase + L::kA1b + sw128_off(r64, d, 8192), pack8_bf16(a));
               }
             }
           }
@@ -916,18 +993,32 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           if (lo16) {
 #pragma unroll
             for (int c8 = 0; c8 < 4; ++c8)
-              st_global_v4(pkg + kPkgA2 + sw128_off(64 + r64, 32 * ch + 8 * c8, 0), pack8_bf16(pt + 8 * c8));
+              st_shared_v4(sbase + L::kA2b + sw128_off(r64, 32 * ch + 8 * c8, 0), pack8_bf16(pt + 8 * c8));
           }
         }
-        // ---- the package is complete: the control warp publishes it ----
+        // ---- the package images are complete: copy them out in bulk; the copies are
+        //      waited for during the next item, then the control warp publishes ----
+        fence_async_smem();
         tc_fence_before();
         cbar();
         tc_fence_after();
-        if (tid == 0) mbar_arrive(&bar_free[b]);
+        if (tid == 0) {
+          bulk_store(pkg + kPkgA1, sm + L::kWm, 8192);
+          bulk_store(pkg + kPkgA1 + 16384, sm + L::kWm + 8192, 8192);
+          bulk_store(pkg + kPkgA1 + 8192, sm + L::kA1b, 8192);
+          bulk_store(pkg + kPkgA1 + 16384 + 8192, sm + L::kA1b + 8192, 8192);
+          bulk_store(pkg + kPkgA2, sm + L::kTu, 8192);
+          bulk_store(pkg + kPkgA2 + 8192, sm + L::kA2b, 8192);
+          bulk_store(pkg + kPkgUs, sm + L::kPv, kPkgCopy - kPkgUs);
+          bulk_commit_group();
+        }
+        out_pending = b;
       }
+      if (tid == 0) finish_out();
     }
   }
 
+  if (tid == 0) bulk_wait_all();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
