@@ -71,10 +71,17 @@ def decode_bytes(B, Hqk, Hv, d):
     return B * Hv * d * d * 4 * 2 + B * Hqk * d * 2 * 2 + B * Hv * d * 2 * 2 + B * Hv * 4 * 2
 
 
-def kernel_source_hash():
+# the source files each kernel is built from (its traffic record is void once one changes)
+KERNEL_SOURCES = {
+    "prefill_pc": ("common.cuh", "sm100.cuh", "prefill_pc.cuh"),
+    "decode": ("common.cuh", "decode.cuh"),
+}
+
+
+def kernel_source_hash(kernel):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_deltanet_linear_21_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
+    for fn in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, fn), "rb") as f:
             h.update(fn.encode() + f.read())
     return h.hexdigest()[:16]
@@ -89,7 +96,7 @@ def traffic_record(kernel):
             rec = json.load(f).get(kernel)
     except (OSError, ValueError):
         return None
-    if not rec or rec.get("source_hash") != kernel_source_hash():
+    if not rec or rec.get("source_hash") != kernel_source_hash(kernel):
         return None
     return rec
 
@@ -159,6 +166,23 @@ class ClockSampler:
                     reasons.add(name)
         return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
                 "reasons": sorted(reasons), "samples": len(self.samples)}
+
+
+def reduce_max(x, world, device=None):
+    """Max over ranks of a host number; every rank calls it at the same point."""
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = device if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_rate(units_per_rank, ms_max, world):
+    """Whole-job rate: every rank processes units_per_rank per step; the job's
+    step time is the slowest rank's."""
+    return world * units_per_rank / (ms_max * 1e-3)
 
 
 def timed(fn, stream):
@@ -341,6 +365,14 @@ def roofline_hbm(nbytes, ms, pk, kind, traffic=None):
             "frac": round(achieved / peak, 4), "traffic": traffic, "peak_kind": f"hbm_gbs ({kind})"}
 
 
+def binding_frac(flops, nbytes, ms, pk):
+    """Fraction of the binding roofline: the larger of the tensor time and the
+    HBM time at the measured peaks, over the measured time."""
+    t_tc = flops / (pk["bf16_tflops"] * 1e12)
+    t_hbm = nbytes / (pk["hbm_gbs"] * 1e9)
+    return round(max(t_tc, t_hbm) / (ms * 1e-3), 4)
+
+
 # -------------------------------------------------------------------- main ---
 def main():
     ap = argparse.ArgumentParser()
@@ -412,12 +444,7 @@ def main():
     pk, pk_kind = peaks()
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        import torch.distributed as dist
-        t = torch.tensor([x], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, world, device)
 
     def barrier():
         if world > 1:
@@ -431,9 +458,9 @@ def main():
         r = run_prefill_bench(gdn, w, args.steps, args.warmup, device, rank, clk)
         barrier()
         ms = max_over_ranks(r["ms"])
-        value = world * r["tokens"] / (ms * 1e-3)
+        value = aggregate_rate(r["tokens"], ms, world)
         flops = prefill_flops_per_token_head(w.chunk, w.d) * r["tokens"] * w.Hv
-        tr = traffic_record("prefill_tc")
+        tr = traffic_record("prefill_pc")
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": DATA,
@@ -441,6 +468,7 @@ def main():
                 "roofline": roofline_tensor(flops, r["ms"], pk, pk_kind,
                                             traffic=tr["bytes_per_launch"] if tr else None),
                 "roofline_hbm_view": roofline_hbm(r["bytes"], r["ms"], pk, pk_kind),
+                "binding_frac": binding_frac(flops, r["bytes"], r["ms"], pk),
                 "gpu_launches": args.steps, "clocks": clk.summary()}
         del r["graph"]
     else:
@@ -450,7 +478,7 @@ def main():
         barrier()
         ms = max_over_ranks(r["ms"])
         tr = traffic_record("decode")
-        line = {"metric": METRIC, "value": world / (ms * 1e-3), "unit": "steps/s", "n_gpus": world,
+        line = {"metric": METRIC, "value": aggregate_rate(1, ms, world), "unit": "steps/s", "n_gpus": world,
                 "steps": r["steps"], "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": DATA,
                 "config": dict(workload_config(w, None, world),
@@ -465,7 +493,7 @@ def main():
         rd = run_decode_bench(gdn, wd, wd.steps, args.warmup, device, rank)
         msd = max_over_ranks(rd["ms"])
         trd = traffic_record("decode")
-        line["decode"] = {"value": world / (msd * 1e-3), "unit": "steps/s", "ms_per_step": msd,
+        line["decode"] = {"value": aggregate_rate(1, msd, world), "unit": "steps/s", "ms_per_step": msd,
                           "steps": rd["steps"], "gpu_launches": rd["steps"],
                           "config": workload_config(wd, None, world),
                           "roofline": roofline_hbm(rd["bytes"], rd["ms"], pk, pk_kind,
@@ -477,16 +505,17 @@ def main():
         del rl["graph"]
         msl = max_over_ranks(rl["ms"])
         fl = prefill_flops_per_token_head(wl.chunk, wl.d) * rl["tokens"] * wl.Hv
-        line["long_prefill"] = {"value": world * rl["tokens"] / (msl * 1e-3), "unit": "tokens/s",
+        line["long_prefill"] = {"value": aggregate_rate(rl["tokens"], msl, world), "unit": "tokens/s",
                                 "ms_per_step": msl, "steps": nl, "gpu_launches": nl,
                                 "config": workload_config(wl, rl["copies"], world),
                                 "roofline": roofline_tensor(fl, rl["ms"], pk, pk_kind),
-                                "roofline_hbm_view": roofline_hbm(rl["bytes"], rl["ms"], pk, pk_kind)}
+                                "roofline_hbm_view": roofline_hbm(rl["bytes"], rl["ms"], pk, pk_kind),
+                                "binding_frac": binding_frac(fl, rl["bytes"], rl["ms"], pk)}
 
     if w.kind == "prefill":
         e = run_e2e(gdn, w, max(3, args.steps // 2), device)
         ems = max_over_ranks(e["ms"])
-        line["e2e"] = {"value": world * e["tokens"] / (ems * 1e-3), "unit": "tokens/s",
+        line["e2e"] = {"value": aggregate_rate(e["tokens"], ems, world), "unit": "tokens/s",
                        "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"]}
     if rank == 0 and world == 1 and not args.no_extras and w.kind == "prefill":
         line["cpu_baseline"] = cpu_baseline(w)

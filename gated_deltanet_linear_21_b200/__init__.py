@@ -16,7 +16,8 @@ import threading
 
 import torch
 
-__all__ = ["prefill", "prefill_noalloc", "decode", "prefill_workspace_bytes", "device_error", "GdnError",
+__all__ = ["prefill", "prefill_noalloc", "decode", "prefill_workspace_bytes", "device_error", "wait_selftest",
+           "GdnError",
            "lib", "library_path", "GDN_BF16", "GDN_F32"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -50,6 +51,7 @@ SIGNATURES = {
     "gdn_prefill_noalloc": (_i, [_vp, _vp, _vp, _fp, _fp, _fp, _i32p, _i, _i64, _i, _i, _i, _i, _f, _i, _i,
                                  _vp, _fp, _vp]),
     "gdn_device_error": (_i, [_vp]),
+    "gdn_wait_selftest": (_i, [_i, _vp]),
 }
 
 
@@ -178,6 +180,12 @@ def decode(q, k, v, g, beta, state, *, scale=None, o=None, stream=None):
         B, Hqk, Hv, dk, dv, float(scale or 0.0), _dtype_code(q), o.data_ptr(),
         _stream_handle(stream)))
     return o
+
+
+def wait_selftest(max_wait_us: int = 2000, stream=None) -> None:
+    """Enqueue the bounded-wait self test (gdn_wait_selftest): a following
+    device_error() raises GdnError with GDN_ERR_DEVICE_TIMEOUT."""
+    _check(lib().gdn_wait_selftest(int(max_wait_us), _stream_handle(stream)))
 
 
 def device_error(stream=None) -> None:

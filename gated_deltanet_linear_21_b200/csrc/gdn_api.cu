@@ -14,7 +14,6 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "prefill_simt.cuh"
-#include "prefill_tc.cuh"
 #include "prefill_pc.cuh"
 
 #include <cudaTypedefs.h>
@@ -144,7 +143,7 @@ bool make_map(CUtensorMap* m, const void* base, int D, int H, int T, int box_d) 
   if (!enc) return false;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T};
   cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
-  cuuint32_t box[3] = {(cuuint32_t)box_d, 1, (cuuint32_t)gdn::tc::kC};
+  cuuint32_t box[3] = {(cuuint32_t)box_d, 1, (cuuint32_t)gdn::pc::kC};
   cuuint32_t estr[3] = {1, 1, 1};
   const int row_bytes = box_d * 2;
   CUtensorMapSwizzle sw = row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
@@ -156,29 +155,6 @@ bool make_map(CUtensorMap* m, const void* base, int D, int H, int T, int box_d) 
   return r == CUDA_SUCCESS;
 }
 
-// Rows of the state per CTA: enough CTAs to cover the 148 SMs once.
-int tc_slice_rows(int n_seqs, int Hv) {
-  if (const char* env = getenv("GDN_TC_SLICE")) {
-    const int v = atoi(env);
-    if (v == 16 || v == 32) return v;
-  }
-  const long chains = (long)n_seqs * Hv;
-  return chains <= 18 ? 16 : 32;
-}
-
-template <int DVP>
-gdn_status launch_tc(const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm, const float* g,
-                     const float* beta, const float* state_in, const int32_t* cu, int n_seqs, int Hqk,
-                     int Hv, float scale, void* o, float* state_out, int total_T, cudaStream_t st) {
-  const size_t smem = gdn::tc::Smem<DVP>::kAlloc;
-  auto kern = gdn::tc::prefill_tc_kernel<DVP>;
-  if (gdn_status s = allow_smem(kern, "gdn_prefill")) return s;
-  dim3 grid(gdn::tc::kD / DVP, (unsigned)Hv, (unsigned)n_seqs);
-  kern<<<grid, gdn::tc::kThreads, smem, st>>>(qm, km, vm, g, beta, state_in, cu, Hqk, Hv, scale,
-                                              static_cast<__nv_bfloat16*>(o), state_out, total_T);
-  return launch_status("gdn_prefill");
-}
-
 int sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -186,8 +162,23 @@ int sm_count() {
   return n;
 }
 
+// The prefill kernel's two bounded waits -- on a ring flag in global memory and
+// on an mbarrier -- each run on something nothing will ever signal, so that the
+// timeout path (error word set, kernel returns) can be exercised without a hung
+// or faulted GPU.
+__device__ uint32_t g_never_set;
+__global__ void wait_selftest_kernel(long long max_cycles) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    gdn::sm100::wait_flag_geq(&g_never_set, 1u, max_cycles);
+    gdn::sm100::mbar_init(&bar, 1);
+    gdn::sm100::fence_mbar_init();
+    gdn::sm100::mbar_wait(&bar, 0, max_cycles);
+  }
+}
+
 bool uses_pc_prefill(gdn_dtype dtype, int dk, int dv) {
-  return dtype == GDN_BF16 && dk == 128 && dv == 128 && !getenv("GDN_PREFILL_FUSED");
+  return dtype == GDN_BF16 && dk == 128 && dv == 128;
 }
 
 template <int DVP>
@@ -289,19 +280,6 @@ gdn_status launch_prefill_pc(const void* q, const void* k, const void* v, const 
   return launch_pc<128>(qm, km, vm, om, prm, sms, st);
 }
 
-gdn_status launch_prefill_tc(const void* q, const void* k, const void* v, const float* g, const float* beta,
-                             const float* state_in, const int32_t* cu, int n_seqs, int64_t total_T, int Hqk,
-                             int Hv, float scale, void* o, float* state_out, cudaStream_t st) {
-  const int dvp = tc_slice_rows(n_seqs, Hv);
-  CUtensorMap qm, km, vm;
-  if (!make_map(&qm, q, 128, Hqk, (int)total_T, 64) || !make_map(&km, k, 128, Hqk, (int)total_T, 64) ||
-      !make_map(&vm, v, 128, Hv, (int)total_T, dvp))
-    return fail(GDN_ERR_CUDA, "gdn_prefill: cuTensorMapEncodeTiled unavailable or failed");
-  if (dvp == 16)
-    return launch_tc<16>(qm, km, vm, g, beta, state_in, cu, n_seqs, Hqk, Hv, scale, o, state_out, (int)total_T, st);
-  return launch_tc<32>(qm, km, vm, g, beta, state_in, cu, n_seqs, Hqk, Hv, scale, o, state_out, (int)total_T, st);
-}
-
 }  // namespace
 
 extern "C" {
@@ -352,9 +330,6 @@ gdn_status gdn_prefill(const void* q, const void* k, const void* v, const float*
   if (uses_pc_prefill(dtype, dk, dv) && C == 64 && total_T > 0)
     return launch_prefill_pc(q, k, v, g, beta, state_in, cu_seqlens, n_seqs, total_T, Hqk, Hv, scale, o, state_out,
                              workspace, st);
-  if (dtype == GDN_BF16 && dk == 128 && dv == 128 && C == 64 && total_T > 0)
-    return launch_prefill_tc(q, k, v, g, beta, state_in, cu_seqlens, n_seqs, total_T, Hqk, Hv, scale, o,
-                             state_out, st);
   if (dtype == GDN_F32)
     return launch_prefill_simt<float>(q, k, v, g, beta, state_in, cu_seqlens, n_seqs, total_T, Hqk,
                                       Hv, dk, dv, scale, C, o, state_out, st);
@@ -385,6 +360,14 @@ gdn_status gdn_decode(const void* q, const void* k, const void* v, const float* 
   if (dtype == GDN_F32)
     return dispatch_decode<float>(q, k, v, g, beta, state, B, Hqk, Hv, dk, dv, scale, o, st);
   return dispatch_decode<__nv_bfloat16>(q, k, v, g, beta, state, B, Hqk, Hv, dk, dv, scale, o, st);
+}
+
+gdn_status gdn_wait_selftest(int max_wait_us, void* stream) {
+  if (max_wait_us < 1 || max_wait_us > 1000000)
+    return fail(GDN_ERR_INVALID_ARG, "gdn_wait_selftest: max_wait_us=%d outside [1, 1000000]", max_wait_us);
+  const long long cycles = (long long)max_wait_us * 2000;   // ~2 GHz SM clock
+  wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(cycles);
+  return launch_status("gdn_wait_selftest");
 }
 
 gdn_status gdn_device_error(void* stream) {

@@ -160,6 +160,19 @@ gdn_status gdn_decode(const void *q, const void *k, const void *v,
                       int B, int Hqk, int Hv, int dk, int dv,
                       float scale, gdn_dtype dtype, void *o, void *stream);
 
+/*
+ * Diagnostic for the failure path, not part of the computation (the pages
+ * have no counterpart). Enqueues one tiny kernel that runs the prefill
+ * kernel's two kinds of bounded wait -- on a flag in global memory and on a
+ * shared-memory mbarrier -- on objects nothing ever signals, each for about
+ * max_wait_us microseconds (1 .. 1000000; ~2 GHz assumed). Both waits run out,
+ * record the timeout in the device error word and return; the kernel ends
+ * normally and the CUDA context stays usable. A following gdn_device_error()
+ * then reports GDN_ERR_DEVICE_TIMEOUT. Returns GDN_ERR_INVALID_ARG for an
+ * out-of-range max_wait_us, GDN_ERR_CUDA if the launch fails.
+ */
+gdn_status gdn_wait_selftest(int max_wait_us, void *stream);
+
 /* Message describing the calling thread's most recent failure ("" if none). */
 const char *gdn_last_error(void);
 
