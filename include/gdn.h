@@ -71,9 +71,15 @@ typedef enum gdn_dtype {
 int gdn_version(void);
 
 /*
- * Bytes of device workspace gdn_prefill needs for this problem (a per-call
- * work list of (sequence, value head, state slice) items ordered longest
- * sequence first, and its counter). Depends only on the arguments given.
+ * Bytes of device workspace gdn_prefill needs for this problem: 0 unless the
+ * tensor-core kernel runs it (GDN_BF16, dk = dv = 128). The tensor-core
+ * kernel splits its CTAs into ones that prepare, per (value head, chunk), the
+ * state-independent operands of the chunk and ones that carry the state from
+ * chunk to chunk; the workspace holds the ring of prepared packages between
+ * them (12 slots of 50 176 bytes per chain running at once, at most 74 chains)
+ * and the ring's flags. It is at most about 44.6 MB however many sequences
+ * there are. Depends only on the arguments given; a call zeroes the flags it
+ * needs, so the contents on entry do not matter.
  */
 size_t gdn_prefill_workspace_bytes(int n_seqs, int Hv, int dk, int dv, gdn_dtype dtype);
 
@@ -96,7 +102,11 @@ size_t gdn_prefill_workspace_bytes(int n_seqs, int Hv, int dk, int dv, gdn_dtype
  *
  * Supported: GDN_BF16 with dk = dv = 128 and chunk 64 (tensor-core kernel);
  * GDN_F32 (and GDN_BF16 with other sizes) with dk, dv in {16, 32, 64, 128}
- * and chunk in {16, 32, 64} (fp32 SIMT kernel). total_T < 2^31.
+ * and chunk in {16, 32, 64} (fp32 SIMT kernel). total_T < 2^31. The
+ * tensor-core kernel runs the sequence-heads in at most 1024 rounds of up to
+ * 74 at a time; larger problems return GDN_ERR_UNSUPPORTED (split them
+ * across calls). It is one cooperative launch with one CTA on every SM of the
+ * device: other work on the device runs before or after it, not beside it.
  * cu_seqlens is read on the device only; a cu_seqlens that breaks the rules
  * above is not detected on the host -- sequences with negative length are
  * treated as empty and tokens past total_T are never read.
@@ -117,14 +127,15 @@ gdn_status gdn_prefill(const void *q, const void *k, const void *v,
  * Herbert pages have no counterpart to it; it exists for integration only.
  *
  * It runs the same tensor-core prefill as gdn_prefill, with the workspace
- * taken from a scratch array compiled into the library (64 MiB of device
- * memory held on every device that loads the library, until the process
- * exits). It calls no allocator. Arguments are those of gdn_prefill without
- * the workspace; the caller still passes every input and output.
+ * taken from a scratch array compiled into the library (45 MiB of device
+ * memory, the largest workspace the kernel can ask for, held on every device
+ * that loads the library until the process exits). It calls no allocator.
+ * Arguments are those of gdn_prefill without the workspace; the caller still
+ * passes every input and output.
  *
- *   Supported: GDN_BF16, dk = dv = 128, chunk 0 or 64. Problems whose workspace
- *   (gdn_prefill_workspace_bytes) exceeds 64 MiB -- more than about 320
- *   sequence-heads -- return GDN_ERR_UNSUPPORTED with a message.
+ *   Supported: GDN_BF16, dk = dv = 128, chunk 0 or 64 (anything else returns
+ *   GDN_ERR_UNSUPPORTED); every problem size gdn_prefill accepts fits the
+ *   array.
  *   The first call on each device looks up the array's device address with
  *   cudaGetSymbolAddress (with that device current); make that first call
  *   before capturing the stream into a CUDA graph.
@@ -152,8 +163,7 @@ gdn_status gdn_prefill_noalloc(const void *q, const void *k, const void *v,
  *   state   [B, Hv, dv, dk]  fp32, updated in place
  *   o       [B, Hv, dv]      dtype (output)
  *
- * Supported: dk = 128 (any dtype), dv any multiple of 8 up to 128... in
- * practice dk in {16, 32, 64, 128} and dv a multiple of 8.
+ * Supported: dk and dv in {16, 32, 64, 128}, either dtype.
  */
 gdn_status gdn_decode(const void *q, const void *k, const void *v,
                       const float *g, const float *beta, float *state,
