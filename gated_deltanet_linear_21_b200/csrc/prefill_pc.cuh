@@ -80,8 +80,9 @@ namespace pc {
 constexpr int kC = 64;
 constexpr int kD = 128;
 constexpr int kCompute = 256;        // compute threads (warps 0-7)
-constexpr int kThreads = 288;        // and the control warp (warp 8)
-constexpr int kCtlWarp = 8;
+constexpr int kThreads = 320;        // and two control warps (8 and 9)
+constexpr int kCtlWarp = 8;          // chain: issues the copies; prep: claims and hands over items
+constexpr int kRelWarp = 9;          // chain: hands ring slots back; prep: publishes packages
 constexpr uint32_t kTmemCols = 512;
 constexpr int kRing = 12;            // package slots per ring position
 constexpr int kMaxRounds = 1024;
@@ -161,8 +162,8 @@ struct Smem {
   static constexpr uint32_t kPrepEnd = kRBase + 4 * (kMaxRounds + 1);
   // common
   static constexpr uint32_t kCommon = ((kChainEnd > kPrepEnd ? kChainEnd : kPrepEnd) + 7) & ~7u;
-  static constexpr uint32_t kBarA = kCommon;                  // full[2], free[2], mma
-  static constexpr uint32_t kMisc = kBarA + 5 * 8;            // tmem slot, scan[4]
+  static constexpr uint32_t kBarA = kCommon;                  // full[2], free[2], mma, pub[2]
+  static constexpr uint32_t kMisc = kBarA + 7 * 8;            // tmem slot, scan[4]
   static constexpr uint32_t kTotal = kMisc + 64;
   static constexpr uint32_t kAlloc = kTotal + 1024;
   static_assert(kAlloc <= 227 * 1024, "shared memory budget");
@@ -231,6 +232,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
   uint64_t* bar_full = reinterpret_cast<uint64_t*>(sm + L::kBarA);  // [2] control -> compute
   uint64_t* bar_free = bar_full + 2;                                 // [2] compute -> control
   uint64_t* bar_mma = bar_full + 4;
+  uint64_t* bar_pub = bar_full + 5;                                  // [2] prep: publisher -> hand-over
   uint32_t* misc = reinterpret_cast<uint32_t*>(sm + L::kMisc);     // [0] tmem, [2..5] scan
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -244,7 +246,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
   const int NC = p.n_chain_ctas;
   const int chains_per_round = NC / kSlices;
   const bool is_chain = (int)blockIdx.x < NC;
-  const bool is_ctl = warp == kCtlWarp;
+  const bool is_ctl = warp == kCtlWarp, is_rel = warp == kRelWarp;
 
   uint32_t* counter = reinterpret_cast<uint32_t*>(p.ws + Workspace::kCounter);
   uint32_t* ready = reinterpret_cast<uint32_t*>(p.ws + Workspace::kFlags);   // [position][slot]
@@ -262,7 +264,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
   };
 
   if (tid == 0) {
-    for (int i = 0; i < 5; ++i) mbar_init(&bar_full[i], 1);
+    for (int i = 0; i < 7; ++i) mbar_init(&bar_full[i], 1);
     fence_mbar_init();
     prefetch_tensormap(&qmap);
     prefetch_tensormap(&kmap);
@@ -310,26 +312,21 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       i0 = (int)(sc % kSlices) * DVP;
       seq_bounds((int)(j / Hv), t_begin, t_end);
     };
+    // the longest chain of the round that chain j belongs to (warp-collective)
+    auto round_maxc = [&](long j, int q) {
+      const long j0 = j - q;
+      int m = 0;
+      for (long jj = j0 + lane; jj < min(j0 + chains_per_round, n_chains); jj += 32) m = max(m, n_chunks_of(jj));
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+      return m;
+    };
+    const int q = (int)blockIdx.x / kSlices;   // ring position (the same in every round)
     if (is_ctl) {
-      // ---- control warp: per chunk, wait for a free buffer and the package's ready
-      //      flag, copy package, k and v in, and hand the ring slot back once landed ----
-      const int q = (int)blockIdx.x / kSlices;   // ring position (the same in every round)
-      uint32_t* rdy = ready + q * kRing;
-      uint32_t* cns = consumed + q * kRing;
+      // ---- issuing warp: per chunk, wait for the package's ready flag and a free input
+      //      buffer, then copy package, k and v in ----
+      const uint32_t* rdy = ready + q * kRing;
       const uint8_t* ring = pkgs + (size_t)q * kRing * kPkgStride;
-      // Copies whose ring slot is not handed back yet, per input buffer (lane 0's
-      // copy of these is the one that counts). A slot goes back as soon as its copy
-      // has landed; the warp never waits for that while it could issue a copy.
-      bool pend[2] = {false, false};
-      int pend_slot[2] = {0, 0};
-      long pend_gc[2] = {0, 0};
-      auto release0 = [&](int bb, bool block) {
-        if (!pend[bb]) return;
-        const uint32_t par = (uint32_t)(pend_gc[bb] >> 1) & 1u;
-        if (block ? !mbar_wait(&bar_full[bb], par) : !mbar_test_wait(&bar_full[bb], par)) return;
-        red_add_release_gpu(&cns[pend_slot[bb]], 1u);
-        pend[bb] = false;
-      };
       long gc = 0;
       int base = 0;
       for (long sc = blockIdx.x; sc < n_slice_chains && !abort; sc += NC) {
@@ -338,32 +335,14 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         decode_sc(sc, j, h, i0, t_begin, t_end);
         const int hq = h / (Hv / Hqk);
         const int nch = (t_end - t_begin + kC - 1) / kC;
-        // the longest chain of this round fixes how many numbers the round takes
-        const long j0 = j - q;
-        int maxc = 0;
-        for (long jj = j0 + lane; jj < min(j0 + chains_per_round, n_chains); jj += 32) maxc = max(maxc, n_chunks_of(jj));
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) maxc = max(maxc, __shfl_xor_sync(0xffffffffu, maxc, off));
+        const int maxc = round_maxc(j, q);
         for (int c = 0; c < nch; ++c, ++gc) {
           const int b = (int)(gc & 1);
           const int s = base + c, slot = s % kRing;
           bool ok = true;
-          if (lane == 0) {   // wait for the package, handing back the other buffer's slot meanwhile
-            const uint32_t want = (uint32_t)(s / kRing + 1);
-            const long long t0 = clock64();
-            while (ld_acquire_gpu(&rdy[slot]) < want) {
-              release0(b ^ 1, false);
-              if (clock64() - t0 > 4000000000ll) {
-                flag_error(kErrTimeout);
-                ok = false;
-                break;
-              }
-              __nanosleep(64);
-            }
-          }
+          if (lane == 0) ok = wait_flag_geq(&rdy[slot], (uint32_t)(s / kRing + 1));
           if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) { abort = true; break; }
           if (gc >= 2 && !mbar_wait(&bar_free[b], (uint32_t)((gc - 2) >> 1) & 1u)) { abort = true; break; }
-          if (lane == 0) release0(b, true);   // (landed: its chunk has been computed)
           fence_async_global();
           uint8_t* dst = sm + L::kIn + b * L::kInBytes;
           const int c0 = t_begin + c * kC;
@@ -374,18 +353,30 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
 #pragma unroll
           for (int vb = 0; vb < L::kBlocks; ++vb)
             tma_load_3d_warp(dst + L::kInV + vb * 64 * L::kRB, &vmap, &bar_full[b], i0 + vb * L::kBlk, h, c0);
-          pend[b] = true;
-          pend_slot[b] = slot;
-          pend_gc[b] = gc;
         }
-        if (abort) break;
-        if (lane == 0)   // numbers this chain leaves unused count as read
-          for (int c = nch; c < maxc; ++c) red_add_release_gpu(&cns[(base + c) % kRing], 1u);
         base += maxc;
       }
-      if (lane == 0) {   // hand back what is still out (bounded waits)
-        release0(0, true);
-        release0(1, true);
+    } else if (is_rel) {
+      // ---- releasing warp: hands each ring slot back once its copy has landed, and
+      //      counts the numbers a shorter chain leaves unused as read ----
+      uint32_t* cns = consumed + q * kRing;
+      long gc = 0;
+      int base = 0;
+      for (long sc = blockIdx.x; sc < n_slice_chains && !abort; sc += NC) {
+        long j;
+        int h, i0, t_begin, t_end;
+        decode_sc(sc, j, h, i0, t_begin, t_end);
+        const int nch = (t_end - t_begin + kC - 1) / kC;
+        const int maxc = round_maxc(j, q);
+        for (int c = 0; c < nch; ++c, ++gc) {
+          // (if this warp is two phases behind, the wait ends with a later copy: only later)
+          if (!mbar_wait(&bar_full[gc & 1], (uint32_t)(gc >> 1) & 1u)) { abort = true; break; }
+          if (lane == 0) red_add_release_gpu(&cns[(base + c) % kRing], 1u);
+        }
+        if (abort) break;
+        if (lane == 0)
+          for (int c = nch; c < maxc; ++c) red_add_release_gpu(&cns[(base + c) % kRing], 1u);
+        base += maxc;
       }
     } else {
       // ---- compute warps ----
@@ -469,21 +460,31 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
               }
             }
           }
-          publish();
-          if (tid == 0 && o_tma) {
-#pragma unroll
-            for (int vb = 0; vb < L::kBlocks; ++vb)
-              tma_store_3d(&omap, in_g + L::kInV + vb * 64 * kRB, i0 + vb * L::kBlk, h, t_begin + c * kC);
-            bulk_commit_group();
-          }
+          // The U warps (0, 1, 4, 5) meet so that warp 0 can issue dS at once; the O
+          // warps (2, 3, 6, 7) only tell warp 0 that their TMEM rows are read and O
+          // is staged, which it needs before the O store and the next chunk's A2 V.
+          fence_async_smem();
+          tc_fence_before();
+          if (qd < 2) named_bar_sync(2, 128);
+          else named_bar_arrive(3, 160);
 
-          // ---- dS^T = K_raw^T U_s ; then, if the next chunk is in, its A2 V ----
+          // ---- dS^T = K_raw^T U_s ; then the O store and, if the next chunk is in, its A2 V ----
           if (warp == 0) {
+            tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               mma_bf16_warp(tmem + kColDS, desc_mnmajor(in + L::kInK, kk, 128, 8192),
                             desc_mnmajor(sUsb, kk, kRB, 64 * kRB), kIdDS, kk > 0);
             mma_commit_warp(bar_mma);
+            named_bar_sync(3, 160);
+            tc_fence_after();
+            if (lane == 0 && o_tma) {
+#pragma unroll
+              for (int vb = 0; vb < L::kBlocks; ++vb)
+                tma_store_3d(&omap, in_g + L::kInV + vb * 64 * kRB, i0 + vb * L::kBlk, h, t_begin + c * kC);
+              bulk_commit_group();
+            }
+            __syncwarp();
             early = false;
             if (c + 1 < nch) {
               const bool nxt = mbar_test_wait(&bar_full[b ^ 1], (uint32_t)((gc + 1) >> 1) & 1u);
@@ -519,44 +520,39 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
   } else {
     // ============================== prep role ===============================
     // round table: items of round r are [round_start[r], round_start[r+1])
-    const long n_rounds = (n_slice_chains + NC - 1) / NC;
-    if (tid == 0) {
-      int acc = 0, nb = 0;
-      for (long r = 0; r < n_rounds && r < kMaxRounds; ++r) {
-        const long j0 = r * chains_per_round;
-        const long j1 = min(j0 + chains_per_round, n_chains);
-        int maxc = 0;
-        for (long jj = j0; jj < j1; ++jj) maxc = max(maxc, n_chunks_of(jj));
-        round_start[r] = acc;
-        rbase[r] = nb;
-        acc += (int)(j1 - j0) * maxc;
-        nb += maxc;
-      }
-      round_start[min(n_rounds, (long)kMaxRounds)] = acc;
+    const int n_rounds = (int)min((n_slice_chains + NC - 1) / NC, (long)kMaxRounds);
+    // the longest chain of each round (warps over rounds, lanes over its chains) ...
+    for (int r = warp; r < n_rounds; r += kThreads / 32) {
+      const long j0 = (long)r * chains_per_round;
+      const long j1 = min(j0 + chains_per_round, n_chains);
+      int maxc = 0;
+      for (long jj = j0 + lane; jj < j1; jj += 32) maxc = max(maxc, n_chunks_of(jj));
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) maxc = max(maxc, __shfl_xor_sync(0xffffffffu, maxc, off));
+      if (lane == 0) rbase[r + 1] = maxc;
     }
     __syncthreads();
-    const int total_items = round_start[min(n_rounds, (long)kMaxRounds)];
+    // ... then the prefix sums: items before round r, numbers before round r
+    if (tid == 0) {
+      int acc = 0, nb = 0;
+      for (int r = 0; r < n_rounds; ++r) {
+        const int maxc = rbase[r + 1];
+        const long j0 = (long)r * chains_per_round;
+        round_start[r] = acc;
+        rbase[r] = nb;
+        acc += (int)(min(j0 + chains_per_round, n_chains) - j0) * maxc;
+        nb += maxc;
+      }
+      round_start[n_rounds] = acc;
+    }
+    __syncthreads();
+    const int total_items = round_start[n_rounds];
 
     if (is_ctl) {
-      // ---- control warp: claim items, fetch gates and raw k, q tiles, wait for the ring
-      //      slot and hand the item over; publish each package once it is written.
-      //      Items are handed over and published in order; at most two are with the
-      //      compute warps. A finished item is published even while the warp waits
-      //      for the slot of a later one (that slot may need this package first). ----
-      int n_handed = 0, n_pub = 0;   // n_pub is advanced by lane 0 and broadcast
-      auto publish0 = [&](bool block) -> bool {   // lane 0: publish item n_pub if its package is written
-        if (n_pub >= n_handed) return false;
-        const int b = n_pub & 1;
-        const uint32_t par = (uint32_t)(n_pub >> 1) & 1u;
-        if (block ? !mbar_wait(&bar_free[b], par) : !mbar_test_wait(&bar_free[b], par)) return false;
-        const uint32_t* qe = reinterpret_cast<const uint32_t*>(sm + L::kQueue + b * L::kQueueBytes);
-        const int s = (int)qe[1], q = (int)qe[2];
-        // the compute warps' package stores precede their barrier and the mbarrier arrival
-        st_release_gpu(&ready[q * kRing + s % kRing], (uint32_t)(s / kRing + 1));
-        ++n_pub;
-        return true;
-      };
-      auto hand_over = [&](int k) -> bool {   // item k -> queue entry k & 1; false once none is left
+      // ---- hand-over warp: claim items, fetch gates and raw k, q tiles, wait for the
+      //      ring slot and hand the item over; queue entry k & 1 is reused once the
+      //      publishing warp has published item k - 2 ----
+      auto hand_over = [&](int k) -> bool {   // false once none is left (or a wait ran out)
         const int b = k & 1;
         uint32_t* qe = reinterpret_cast<uint32_t*>(sm + L::kQueue + b * L::kQueueBytes);
         int v = 0, c = 0, q = 0, s = 0;
@@ -565,8 +561,12 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           while (true) {
             const int item = (int)atomicAdd(counter, 1u);
             if (item >= total_items) break;
-            int r = 0;
-            while (round_start[r + 1] <= item) ++r;
+            int r = 0, hi = n_rounds - 1;   // the round holding the item
+            while (r < hi) {
+              const int mid = (r + hi + 1) >> 1;
+              if (round_start[mid] <= item) r = mid;
+              else hi = mid - 1;
+            }
             const long j0 = (long)r * chains_per_round;
             const int cpr = (int)(min(j0 + chains_per_round, n_chains) - j0);
             const int local = item - round_start[r];
@@ -597,22 +597,8 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             qg[e] = e < len ? p.g[(size_t)(c0 + e) * Hv + h] : 0.f;
             qb[e] = e < len ? p.beta[(size_t)(c0 + e) * Hv + h] : 0.f;
           }
-          if (lane == 0) {   // wait for the ring slot, publishing finished items meanwhile
-            const uint32_t* flag = &consumed[q * kRing + s % kRing];
-            const uint32_t want = (uint32_t)(kSlices * (s / kRing));
-            const long long t0 = clock64();
-            while (ld_acquire_gpu(flag) < want) {
-              publish0(false);
-              if (clock64() - t0 > 4000000000ll) {
-                flag_error(kErrTimeout);
-                ok = false;
-                break;
-              }
-              __nanosleep(64);
-            }
-          }
+          if (lane == 0) ok = wait_flag_geq(&consumed[q * kRing + s % kRing], (uint32_t)(kSlices * (s / kRing)));
           ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-          n_pub = __shfl_sync(0xffffffffu, n_pub, 0);
         }
         const bool go = v && ok;
         if (lane == 0) {
@@ -635,19 +621,23 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         }
         return go;
       };
-      bool ended = false;
-      while (true) {
-        if (!ended && n_handed - n_pub < 2) {   // a queue entry is free
-          if (hand_over(n_handed)) ++n_handed;
-          else ended = true;
-        } else if (n_pub < n_handed) {
-          bool ok = true;
-          if (lane == 0) ok = publish0(true);
-          if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
-          n_pub = __shfl_sync(0xffffffffu, n_pub, 0);
-        } else {
-          break;
-        }
+      for (int k = 0;; ++k) {
+        if (k >= 2 && !mbar_wait(&bar_pub[k & 1], (uint32_t)((k - 2) >> 1) & 1u)) break;
+        if (!hand_over(k)) break;
+      }
+    } else if (is_rel) {
+      // ---- publishing warp: once the compute warps have written item `it`'s package
+      //      (their bulk copies complete and fenced), release its ready flag ----
+      for (int it = 0;; ++it) {
+        const int b = it & 1;
+        const uint32_t par = (uint32_t)(it >> 1) & 1u;
+        if (!mbar_wait(&bar_full[b], par)) break;   // handed over (or the end marker)
+        const uint32_t* qe = reinterpret_cast<const uint32_t*>(sm + L::kQueue + b * L::kQueueBytes);
+        if (qe[0] == 0) break;
+        if (!mbar_wait(&bar_free[b], par)) break;
+        if (lane == 0) st_release_gpu(&ready[qe[2] * kRing + qe[1] % kRing], qe[1] / kRing + 1);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_pub[b]);
       }
     } else {
       // ---- compute warps ----

@@ -87,6 +87,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
+// Arrives on barrier `id` (counted among its `n` threads) without waiting.
+__device__ __forceinline__ void named_bar_arrive(int id, int n) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
 // As named_bar_sync, and returns whether `p` holds on every participating thread.
 __device__ __forceinline__ bool named_bar_and(int id, int n, bool p) {
   uint32_t r;
