@@ -80,9 +80,10 @@ namespace pc {
 constexpr int kC = 64;
 constexpr int kD = 128;
 constexpr int kCompute = 256;        // compute threads (warps 0-7)
-constexpr int kThreads = 320;        // and two control warps (8 and 9)
+constexpr int kThreads = 352;        // and three warps with their own jobs:
 constexpr int kCtlWarp = 8;          // chain: issues the copies; prep: claims and hands over items
 constexpr int kRelWarp = 9;          // chain: hands ring slots back; prep: publishes packages
+constexpr int kMmaWarp = 10;         // chain: issues the tensor-core work and the O store
 constexpr uint32_t kTmemCols = 512;
 constexpr int kRing = 12;            // package slots per ring position
 constexpr int kMaxRounds = 1024;
@@ -162,8 +163,8 @@ struct Smem {
   static constexpr uint32_t kPrepEnd = kRBase + 4 * (kMaxRounds + 1);
   // common
   static constexpr uint32_t kCommon = ((kChainEnd > kPrepEnd ? kChainEnd : kPrepEnd) + 7) & ~7u;
-  static constexpr uint32_t kBarA = kCommon;                  // full[2], free[2], mma, pub[2]
-  static constexpr uint32_t kMisc = kBarA + 7 * 8;            // tmem slot, scan[4]
+  static constexpr uint32_t kBarA = kCommon;                  // full[2], free[2], mma, pub[2] | u, o, s
+  static constexpr uint32_t kMisc = kBarA + 8 * 8;            // tmem slot, scan[4]
   static constexpr uint32_t kTotal = kMisc + 64;
   static constexpr uint32_t kAlloc = kTotal + 1024;
   static_assert(kAlloc <= 227 * 1024, "shared memory budget");
@@ -233,6 +234,9 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
   uint64_t* bar_free = bar_full + 2;                                 // [2] compute -> control
   uint64_t* bar_mma = bar_full + 4;
   uint64_t* bar_pub = bar_full + 5;                                  // [2] prep: publisher -> hand-over
+  uint64_t* bar_u = bar_full + 5;      // chain: U_s staged (the 4 U warps)
+  uint64_t* bar_o = bar_full + 6;      // chain: O staged (the 4 O warps)
+  uint64_t* bar_s = bar_full + 7;      // chain: the bf16 state copy is written
   uint32_t* misc = reinterpret_cast<uint32_t*>(sm + L::kMisc);     // [0] tmem, [2..5] scan
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -264,7 +268,13 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
   };
 
   if (tid == 0) {
-    for (int i = 0; i < 7; ++i) mbar_init(&bar_full[i], 1);
+    // chain: a buffer is free once the compute warps and the MMA warp are done with
+    // it; U_s and O are staged by four warps each
+    for (int i = 0; i < 8; ++i) {
+      const bool two = is_chain && (i == 2 || i == 3);
+      const bool four = is_chain && (i == 5 || i == 6);
+      mbar_init(&bar_full[i], two ? 2 : four ? 4 : 1);
+    }
     fence_mbar_init();
     prefetch_tensormap(&qmap);
     prefetch_tensormap(&kmap);
@@ -343,6 +353,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           if (lane == 0) ok = wait_flag_geq(&rdy[slot], (uint32_t)(s / kRing + 1));
           if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) { abort = true; break; }
           if (gc >= 2 && !mbar_wait(&bar_free[b], (uint32_t)((gc - 2) >> 1) & 1u)) { abort = true; break; }
+          __syncwarp();
           fence_async_global();
           uint8_t* dst = sm + L::kIn + b * L::kInBytes;
           const int c0 = t_begin + c * kC;
@@ -378,107 +389,59 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           for (int c = nch; c < maxc; ++c) red_add_release_gpu(&cns[(base + c) % kRing], 1u);
         base += maxc;
       }
-    } else {
-      // ---- compute warps ----
+    } else if (warp == kMmaWarp || warp < 8) {
       constexpr uint32_t kIdY = idesc_bf16(128, DVP, false, true);
       constexpr uint32_t kIdDS = idesc_bf16(128, DVP, true, true);
       const uint32_t sSb = sbase + L::kSb;
       const uint32_t sUsb = sbase + L::kUsb;
-      // A2 V_raw of input buffer b into Y, as the first term (warp 0)
-      auto issue_a2v = [&](int b) {
-        const uint32_t in = sbase + L::kIn + b * L::kInBytes;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16_warp(tmem + kColY, desc_kmajor(in + kPkgA2, kk, 0), desc_mnmajor(in + L::kInV, kk, kRB, 64 * kRB),
-                        kIdY, kk > 0);
-      };
-      long gc = 0;
-      bool early = false;   // (warp 0) A2 V of the current chunk is already issued
-      for (long sc = blockIdx.x; sc < n_slice_chains && !abort; sc += NC) {
-        long j;
-        int h, i0, t_begin, t_end;
-        decode_sc(sc, j, h, i0, t_begin, t_end);
-        const int n = (int)(j / Hv);
-        const int nch = (t_end - t_begin + kC - 1) / kC;
-
-        const size_t s_off = ((size_t)n * Hv + h) * kD * kD + (size_t)(i0 + ch * kHalf) * kD + r128;
-        float Sreg[kHalf];
-#pragma unroll
-        for (int q2 = 0; q2 < kHalf; ++q2) Sreg[q2] = p.state_in ? p.state_in[s_off + (size_t)q2 * kD] : 0.f;
-        auto store_state = [&]() {
-#pragma unroll
-          for (int c8 = 0; c8 < kHalf / 8; ++c8)
-            st_shared_v4(sSb + L::tile_off(r128, ch * kHalf + 8 * c8, 128), pack8_bf16(Sreg + 8 * c8));
-        };
-        store_state();
-        publish();
-
-        for (int c = 0; c < nch; ++c, ++gc) {
-          const int b = (int)(gc & 1);
+      if (warp == kMmaWarp) {
+        // ---- MMA warp: per chunk Y = A2 V + A1 S^T (rows 0-63 U, rows 64-127 O), then
+        //      dS^T = K_raw^T U_s, the O store, and the next chunk's A2 V when its data
+        //      is in; it waits on the compute warps through mbarriers (bounded) ----
+        auto issue_a2v = [&](int b) {   // A2 V_raw of input buffer b, the first term of Y
           const uint32_t in = sbase + L::kIn + b * L::kInBytes;
-          const uint8_t* in_g = sm + L::kIn + b * L::kInBytes;
-          const bool full_ok = mbar_wait(&bar_full[b], (uint32_t)(gc >> 1) & 1u);
-          const int len = min(kC, t_end - (t_begin + c * kC));
-
-          // ---- Y = A2 V + A1 S^T : rows 0-63 U, rows 64-127 O ----
-          if (warp == 0) {
-            if (full_ok) {
-              if (!early) issue_a2v(b);
 #pragma unroll
-              for (int kk = 0; kk < 8; ++kk)
-                mma_bf16_warp(tmem + kColY, desc_kmajor(in + kPkgA1, kk, 16384), desc_mnmajor(sSb, kk, kRB, 128 * kRB),
-                              kIdY, 1u);
-            }
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_warp(tmem + kColY, desc_kmajor(in + kPkgA2, kk, 0), desc_mnmajor(in + L::kInV, kk, kRB, 64 * kRB),
+                          kIdY, kk > 0);
+        };
+        long gc = 0;
+        bool early = false;
+        uint32_t ph_u = 0, ph_o = 0, ph_s = 0;
+        for (long sc = blockIdx.x; sc < n_slice_chains && !abort; sc += NC) {
+          long j;
+          int h, i0, t_begin, t_end;
+          decode_sc(sc, j, h, i0, t_begin, t_end);
+          const int nch = (t_end - t_begin + kC - 1) / kC;
+          for (int c = 0; c < nch; ++c, ++gc) {
+            const int b = (int)(gc & 1);
+            const uint32_t in = sbase + L::kIn + b * L::kInBytes;
+            const uint8_t* in_g = sm + L::kIn + b * L::kInBytes;
+            const bool o_tma = t_end - (t_begin + c * kC) >= kC;
+            if (!mbar_wait(&bar_full[b], (uint32_t)(gc >> 1) & 1u) || !mbar_wait(bar_s, ph_s)) { abort = true; break; }
+            ph_s ^= 1;
+            __syncwarp();
+            tc_fence_after();
+            if (!early) issue_a2v(b);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_bf16_warp(tmem + kColY, desc_kmajor(in + kPkgA1, kk, 16384), desc_mnmajor(sSb, kk, kRB, 128 * kRB),
+                            kIdY, 1u);
             mma_commit_warp(bar_mma);
-          }
-          if (!wait_mma(full_ok)) { abort = true; break; }
-          // O of a whole chunk goes out by TMA from the v tile's place (v is consumed);
-          // the rows of a sequence's last, partial chunk are stored one by one
-          const bool o_tma = len == kC;
-          {
-            const float us = qd < 2 ? reinterpret_cast<const float*>(in_g + kPkgUs)[r128] : 0.f;
-            __nv_bfloat16* orow = p.o + ((size_t)(t_begin + c * kC + (r128 & 63)) * Hv + h) * kD + i0 + ch * kHalf;
-#pragma unroll
-            for (int pp = 0; pp < kHalf / kPart; ++pp) {
-              float yv[kPart];
-              tmem_ld<kPart>(tmem + tlane + kColY + ch * kHalf + pp * kPart, yv);
-              if (qd < 2) {   // U_s = diag(us) U -> shared memory (bf16) for dS
-#pragma unroll
-                for (int q2 = 0; q2 < kPart; ++q2) yv[q2] *= us;
-#pragma unroll
-                for (int c8 = 0; c8 < kPart / 8; ++c8)
-                  st_shared_v4(sUsb + L::tile_off(r128, ch * kHalf + pp * kPart + 8 * c8, 64), pack8_bf16(yv + 8 * c8));
-              } else if (o_tma) {
-#pragma unroll
-                for (int c8 = 0; c8 < kPart / 8; ++c8)
-                  st_shared_v4(in + L::kInV + L::tile_off(r128 - 64, ch * kHalf + pp * kPart + 8 * c8, 64),
-                               pack8_bf16(yv + 8 * c8));
-              } else if (r128 - 64 < len) {
-#pragma unroll
-                for (int c8 = 0; c8 < kPart / 8; ++c8)
-                  *reinterpret_cast<uint4*>(orow + pp * kPart + 8 * c8) = pack8_bf16(yv + 8 * c8);
-              }
-            }
-          }
-          // The U warps (0, 1, 4, 5) meet so that warp 0 can issue dS at once; the O
-          // warps (2, 3, 6, 7) only tell warp 0 that their TMEM rows are read and O
-          // is staged, which it needs before the O store and the next chunk's A2 V.
-          fence_async_smem();
-          tc_fence_before();
-          if (qd < 2) named_bar_sync(2, 128);
-          else named_bar_arrive(3, 160);
-
-          // ---- dS^T = K_raw^T U_s ; then the O store and, if the next chunk is in, its A2 V ----
-          if (warp == 0) {
+            if (!mbar_wait(bar_u, ph_u)) { abort = true; break; }
+            ph_u ^= 1;
+            __syncwarp();
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               mma_bf16_warp(tmem + kColDS, desc_mnmajor(in + L::kInK, kk, 128, 8192),
                             desc_mnmajor(sUsb, kk, kRB, 64 * kRB), kIdDS, kk > 0);
             mma_commit_warp(bar_mma);
-            named_bar_sync(3, 160);
+            if (!mbar_wait(bar_o, ph_o)) { abort = true; break; }
+            ph_o ^= 1;
+            __syncwarp();
             tc_fence_after();
-            if (lane == 0 && o_tma) {
+            if (lane == 0 && o_tma) {   // O of a whole chunk goes out from the v tile's place
 #pragma unroll
               for (int vb = 0; vb < L::kBlocks; ++vb)
                 tma_store_3d(&omap, in_g + L::kInV + vb * 64 * kRB, i0 + vb * L::kBlk, h, t_begin + c * kC);
@@ -493,28 +456,100 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
                 early = true;
               }
             }
-          }
-          if (!wait_mma()) { abort = true; break; }
-          {
-            const float gL = *reinterpret_cast<const float*>(in_g + kPkgGL);
-#pragma unroll
-            for (int pp = 0; pp < kHalf / kPart; ++pp) {
-              float ds[kPart];
-              tmem_ld<kPart>(tmem + tlane + kColDS + ch * kHalf + pp * kPart, ds);
-#pragma unroll
-              for (int q2 = 0; q2 < kPart; ++q2) Sreg[pp * kPart + q2] = fmaf(gL, Sreg[pp * kPart + q2], ds[q2]);
+            if (lane == 0) {
+              bulk_wait_read_all();   // the O tile has left the buffer
+              mbar_arrive(&bar_free[b]);
             }
-            store_state();
-          }
-          publish();
-          if (tid == 0) {
-            bulk_wait_read_all();   // the O tile has left the buffer
-            mbar_arrive(&bar_free[b]);
+            __syncwarp();
           }
         }
-        if (abort) break;
+      } else {
+        // ---- compute warps: the Y and dS epilogues and the fp32 state ----
+        long gc = 0;
+        auto warp_arrive = [&](uint64_t* bar) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar);
+        };
+        for (long sc = blockIdx.x; sc < n_slice_chains && !abort; sc += NC) {
+          long j;
+          int h, i0, t_begin, t_end;
+          decode_sc(sc, j, h, i0, t_begin, t_end);
+          const int n = (int)(j / Hv);
+          const int nch = (t_end - t_begin + kC - 1) / kC;
+
+          const size_t s_off = ((size_t)n * Hv + h) * kD * kD + (size_t)(i0 + ch * kHalf) * kD + r128;
+          float Sreg[kHalf];
 #pragma unroll
-        for (int q2 = 0; q2 < kHalf; ++q2) p.state_out[s_off + (size_t)q2 * kD] = Sreg[q2];
+          for (int q2 = 0; q2 < kHalf; ++q2) Sreg[q2] = p.state_in ? p.state_in[s_off + (size_t)q2 * kD] : 0.f;
+          auto store_state = [&]() {
+#pragma unroll
+            for (int c8 = 0; c8 < kHalf / 8; ++c8)
+              st_shared_v4(sSb + L::tile_off(r128, ch * kHalf + 8 * c8, 128), pack8_bf16(Sreg + 8 * c8));
+          };
+          if (nch > 0) {
+            store_state();
+            publish();
+            if (tid == 0) mbar_arrive(bar_s);
+          }
+
+          for (int c = 0; c < nch; ++c, ++gc) {
+            const int b = (int)(gc & 1);
+            const uint32_t in = sbase + L::kIn + b * L::kInBytes;
+            const uint8_t* in_g = sm + L::kIn + b * L::kInBytes;
+            const bool full_ok = mbar_wait(&bar_full[b], (uint32_t)(gc >> 1) & 1u);
+            const int len = min(kC, t_end - (t_begin + c * kC));
+            const bool o_tma = len == kC;
+            if (!wait_mma(full_ok)) { abort = true; break; }   // Y
+            {
+              const float us = qd < 2 ? reinterpret_cast<const float*>(in_g + kPkgUs)[r128] : 0.f;
+              __nv_bfloat16* orow = p.o + ((size_t)(t_begin + c * kC + (r128 & 63)) * Hv + h) * kD + i0 + ch * kHalf;
+#pragma unroll
+              for (int pp = 0; pp < kHalf / kPart; ++pp) {
+                float yv[kPart];
+                tmem_ld<kPart>(tmem + tlane + kColY + ch * kHalf + pp * kPart, yv);
+                if (qd < 2) {   // U_s = diag(us) U -> shared memory (bf16) for dS
+#pragma unroll
+                  for (int q2 = 0; q2 < kPart; ++q2) yv[q2] *= us;
+#pragma unroll
+                  for (int c8 = 0; c8 < kPart / 8; ++c8)
+                    st_shared_v4(sUsb + L::tile_off(r128, ch * kHalf + pp * kPart + 8 * c8, 64), pack8_bf16(yv + 8 * c8));
+                } else if (o_tma) {   // O staged in the consumed v tile for the TMA store
+#pragma unroll
+                  for (int c8 = 0; c8 < kPart / 8; ++c8)
+                    st_shared_v4(in + L::kInV + L::tile_off(r128 - 64, ch * kHalf + pp * kPart + 8 * c8, 64),
+                                 pack8_bf16(yv + 8 * c8));
+                } else if (r128 - 64 < len) {   // a sequence's last, partial chunk: row by row
+#pragma unroll
+                  for (int c8 = 0; c8 < kPart / 8; ++c8)
+                    *reinterpret_cast<uint4*>(orow + pp * kPart + 8 * c8) = pack8_bf16(yv + 8 * c8);
+                }
+              }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            warp_arrive(qd < 2 ? bar_u : bar_o);
+            if (!wait_mma()) { abort = true; break; }   // dS
+            {
+              const float gL = *reinterpret_cast<const float*>(in_g + kPkgGL);
+#pragma unroll
+              for (int pp = 0; pp < kHalf / kPart; ++pp) {
+                float ds[kPart];
+                tmem_ld<kPart>(tmem + tlane + kColDS + ch * kHalf + pp * kPart, ds);
+#pragma unroll
+                for (int q2 = 0; q2 < kPart; ++q2) Sreg[pp * kPart + q2] = fmaf(gL, Sreg[pp * kPart + q2], ds[q2]);
+              }
+              store_state();
+            }
+            publish();
+            if (tid == 0) {
+              if (c + 1 < nch) mbar_arrive(bar_s);
+              mbar_arrive(&bar_free[b]);
+            }
+          }
+          if (abort) break;
+#pragma unroll
+          for (int q2 = 0; q2 < kHalf; ++q2) p.state_out[s_off + (size_t)q2 * kD] = Sreg[q2];
+        }
       }
     }
   } else {
@@ -623,6 +658,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       };
       for (int k = 0;; ++k) {
         if (k >= 2 && !mbar_wait(&bar_pub[k & 1], (uint32_t)((k - 2) >> 1) & 1u)) break;
+        __syncwarp();
         if (!hand_over(k)) break;
       }
     } else if (is_rel) {
@@ -639,8 +675,8 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar_pub[b]);
       }
-    } else {
-      // ---- compute warps ----
+    } else if (warp < 8) {
+      // ---- compute warps (warp 10 has no job in a prep CTA) ----
       constexpr uint32_t kIdG = idesc_bf16(128, 64, false, false);
       constexpr uint32_t kId64 = idesc_bf16(64, 64, false, true);
       constexpr uint32_t kIdW = idesc_bf16(64, 128, false, true);
