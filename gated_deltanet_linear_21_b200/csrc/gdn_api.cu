@@ -211,8 +211,8 @@ struct PcPlan {
   long nc;
 };
 PcPlan plan_pc(long chains, int64_t total_T, int n_seqs, int sms) {
-  const double kChainStep[3] = {2300.0, 2800.0, 3600.0};   // DVP 32, 64, 128
-  const double kPrepItem = 12700.0;
+  const double kChainStep[3] = {2200.0, 2600.0, 3400.0};   // DVP 32, 64, 128
+  const double kPrepItem = 10300.0;
   const double chunks = std::max(1.0, std::ceil((double)total_T / std::max(1, n_seqs) / 64.0));
   PcPlan best = {128, 1};
   double best_t = 1e300;

@@ -118,9 +118,9 @@ constexpr uint32_t kColG = 0;      // prep: [k;q] k^T       M=128, N=64
 constexpr uint32_t kColN = 64;     // prep: N = D A_o       M=64 (lanes 0-15)
 constexpr uint32_t kColS2 = 128;   // prep: N D (lanes 0-15), N^2 (lanes 16-31)
 constexpr uint32_t kColZ = 192;    // prep: N^2 E           M=64
-constexpr uint32_t kColW = 256;    // prep: -W              M=64, N=128
-constexpr uint32_t kColPW = 384;   // prep: -P W            M=64, N=128
-constexpr uint32_t kColPT = 0;     // prep: P T_u           M=64, N=64 (Gram columns, free by then)
+constexpr uint32_t kColW = 256;    // prep: -W, d_k 0-63 in lanes 0-15, 64-127 in lanes 16-31
+constexpr uint32_t kColPW = 320;   // prep: -P W, the same split
+constexpr uint32_t kColPT = 384;   // prep: P T_u           M=64, N=64 (lanes 0-15)
 constexpr uint32_t kColY = 0;      // chain: Y = [U ; O]    M=128, N=DVP
 constexpr uint32_t kColDS = 128;   // chain: dS^T           M=128, N=DVP
 
@@ -679,7 +679,6 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       // ---- compute warps (warp 10 has no job in a prep CTA) ----
       constexpr uint32_t kIdG = idesc_bf16(128, 64, false, false);
       constexpr uint32_t kId64 = idesc_bf16(64, 64, false, true);
-      constexpr uint32_t kIdW = idesc_bf16(64, 128, false, true);
       float* vG = reinterpret_cast<float*>(sm + L::kVec);   // per-warp partial scan of g
       float* vB = vG + 64;
       float* vRk = vB + 64;
@@ -957,25 +956,27 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         }
         publish();
 
-        // ---- -W = (-T_w) K_raw -> shared (operand of P W) and the package (A1 rows 0-63) ----
+        // ---- -W = (-T_w) K_raw -> shared (operand of P W and A1 rows 0-63); the two
+        //      column halves go to the two lane halves so that every thread has work ----
+        const int dhalf = 64 * (lane >> 4) + 32 * ch;   // this thread's 32 columns of a d_k-wide row
         if (warp == 0) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_warp(tmem + kColW, desc_kmajor(sbase + L::kTw, kk, 0), desc_mnmajor(sKQ, kk, 128, 16384), kIdW,
+            mma_bf16_warp(tmem + kColW, desc_kmajor(sbase + L::kTw, kk, 0), desc_mnmajor(sKQ, kk, 128, 16384), kId64,
                           kk > 0);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_warp(tmem + (16u << 16) + kColW, desc_kmajor(sbase + L::kTw, kk, 0),
+                          desc_mnmajor(sKQ + 16384, kk, 128, 16384), kId64, kk > 0);
           mma_commit_warp(bar_mma);
         }
         if (!wait_mma()) { abort = true; break; }
         {
-          float w[64];
-          tmem_ld64(tmem + tlane + kColW + 64 * ch, w);
-          if (lo16) {
+          float w[32];
+          tmem_ld32(tmem + tlane + kColW + 32 * ch, w);
 #pragma unroll
-            for (int c8 = 0; c8 < 8; ++c8) {
-              const int d = 64 * ch + 8 * c8;
-              st_shared_v4(sbase + L::kWm + sw128_off(r64, d, 8192), pack8_bf16(w + 8 * c8));
-            }
-          }
+          for (int c8 = 0; c8 < 4; ++c8)
+            st_shared_v4(sbase + L::kWm + sw128_off(r64, dhalf + 8 * c8, 8192), pack8_bf16(w + 8 * c8));
         }
         publish();
 
@@ -984,7 +985,11 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_bf16_warp(tmem + kColPW, desc_kmajor(sbase + L::kPm, kk, 0), desc_mnmajor(sbase + L::kWm, kk, 128, 8192),
-                          kIdW, kk > 0);
+                          kId64, kk > 0);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_warp(tmem + (16u << 16) + kColPW, desc_kmajor(sbase + L::kPm, kk, 0),
+                          desc_mnmajor(sbase + L::kWm + 8192, kk, 128, 8192), kId64, kk > 0);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_bf16_warp(tmem + kColPT, desc_kmajor(sbase + L::kPm, kk, 0), desc_mnmajor(sbase + L::kTu, kk, 128, 8192),
@@ -995,23 +1000,21 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         {
           const float rho = vRho[r64];
           {
-            float pw[64];
-            tmem_ld64(tmem + tlane + kColPW + 64 * ch, pw);
-            if (lo16) {
+            float pw[32];
+            tmem_ld32(tmem + tlane + kColPW + 32 * ch, pw);
 #pragma unroll
-              for (int c8 = 0; c8 < 8; ++c8) {
-                const int d = 64 * ch + 8 * c8;
-                const uint4 qv = ld_shared_v4(sKQ + sw128_off(64 + r64, d, 16384));
-                const __nv_bfloat162* q2v = reinterpret_cast<const __nv_bfloat162*>(&qv);
-                float a[8];
+            for (int c8 = 0; c8 < 4; ++c8) {
+              const int d = dhalf + 8 * c8;
+              const uint4 qv = ld_shared_v4(sKQ + sw128_off(64 + r64, d, 16384));
+              const __nv_bfloat162* q2v = reinterpret_cast<const __nv_bfloat162*>(&qv);
+              float a[8];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const float2 qf = __bfloat1622float2(q2v[e]);
-                  a[2 * e] = fmaf(rho, qf.x, pw[8 * c8 + 2 * e]);
-                  a[2 * e + 1] = fmaf(rho, qf.y, pw[8 * c8 + 2 * e + 1]);
-                }
-                st_shared_v4(sbase + L::kA1b + sw128_off(r64, d, 8192), pack8_bf16(a));
+              for (int e = 0; e < 4; ++e) {
+                const float2 qf = __bfloat1622float2(q2v[e]);
+                a[2 * e] = fmaf(rho, qf.x, pw[8 * c8 + 2 * e]);
+                a[2 * e + 1] = fmaf(rho, qf.y, pw[8 * c8 + 2 * e + 1]);
               }
+              st_shared_v4(sbase + L::kA1b + sw128_off(r64, d, 8192), pack8_bf16(a));
             }
           }
           float pt[32];
