@@ -498,6 +498,15 @@ def main():
                           "config": workload_config(wd, None, world),
                           "roofline": roofline_hbm(rd["bytes"], rd["ms"], pk, pk_kind,
                                                    traffic=trd["bytes_per_launch"] if trd else None)}
+        # one request at a time: B=1 decode, 1000 steps in one CUDA graph
+        wb = workloads.Workload("decode_b1", 2, "decode", batch=1, steps=1000, Hqk=16, Hv=32,
+                                state_std=wd.state_std)
+        rb = run_decode_bench(gdn, wb, wb.steps, args.warmup, device, rank)
+        msb = max_over_ranks(rb["ms"])
+        line["decode_b1"] = {"value": aggregate_rate(1, msb, world), "unit": "steps/s", "ms_per_step": msb,
+                             "steps": rb["steps"], "gpu_launches": rb["steps"],
+                             "config": workload_config(wb, None, world),
+                             "roofline": roofline_hbm(rb["bytes"], rb["ms"], pk, pk_kind)}
         # long prompt: 32768 tokens, 16 q/k and 32 v heads
         wl = workloads.workload("long")
         nl = max(2, args.steps // 4)

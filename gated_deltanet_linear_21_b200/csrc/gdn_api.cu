@@ -202,15 +202,19 @@ gdn_status launch_pc(const CUtensorMap& qm, const CUtensorMap& km, const CUtenso
 }
 
 // Chooses the state slice width DVP and the number of chain CTAs. The kernel
-// runs min(NC, slice-chains) state chains at a time, in rounds, and prepares
-// packages on the remaining CTAs; its time is about the larger of the two
-// sides. Per-chunk costs (SM cycles) measured on B200: a chain step of one
-// slice and the preparation of one (head, chunk) item.
+// runs P = NC / slices chains (sequence-heads) at a time, in rounds, and
+// prepares packages on the remaining CTAs; its time is about the larger of the
+// two sides. Per-chunk costs (SM cycles) measured on B200: a chain step of one
+// slice and the preparation of one (head, chunk) item. With several sequences a
+// round lasts as long as its longest chain, so P is kept to a multiple or a
+// divisor of Hv (whole sequences, or equal parts of one, per round) and a round
+// of m sequences is charged the expected longest of m: 2m / (m + 1) times the
+// mean length (the lengths are on the device; only their mean is known here).
 struct PcPlan {
   int dvp;
   long nc;
 };
-PcPlan plan_pc(long chains, int64_t total_T, int n_seqs, int sms) {
+PcPlan plan_pc(long chains, int64_t total_T, int n_seqs, int Hv, int sms) {
   const double kChainStep[3] = {2200.0, 2600.0, 3400.0};   // DVP 32, 64, 128
   const double kPrepItem = 10300.0;
   const double chunks = std::max(1.0, std::ceil((double)total_T / std::max(1, n_seqs) / 64.0));
@@ -218,10 +222,17 @@ PcPlan plan_pc(long chains, int64_t total_T, int n_seqs, int sms) {
   double best_t = 1e300;
   for (int t = 0; t < 3; ++t) {
     const int dvp = 32 << t, slices = 128 / dvp;
-    const long nc_max = std::min({chains * slices, (long)gdn::pc::kMaxPositions * slices, (long)sms - 8});
-    for (long nc = slices; nc <= nc_max; nc += slices) {
-      const double rounds = std::ceil((double)(chains * slices) / nc);
-      const double chain_t = rounds * chunks * kChainStep[t];
+    const long p_max = std::min({chains, (long)gdn::pc::kMaxPositions, ((long)sms - 8) / slices});
+    for (long pos = 1; pos <= p_max; ++pos) {
+      double maxf = 1.0;
+      if (n_seqs > 1) {
+        if (pos % Hv != 0 && Hv % pos != 0) continue;
+        const double m = pos >= Hv ? (double)(pos / Hv) : 1.0;
+        maxf = 2.0 * m / (m + 1.0);
+      }
+      const long nc = pos * slices;
+      const double rounds = std::ceil((double)chains / pos);
+      const double chain_t = rounds * chunks * maxf * kChainStep[t];
       const double prep_t = chains * chunks * kPrepItem / (double)(sms - nc);
       const double tt = std::max(chain_t, prep_t);
       if (tt < best_t * 0.999) {
@@ -239,7 +250,7 @@ gdn_status launch_prefill_pc(const void* q, const void* k, const void* v, const 
   const long chains = (long)n_seqs * Hv;
   const int sms = sm_count();
   if (sms < 16) return fail(GDN_ERR_CUDA, "gdn_prefill: cannot query the multiprocessor count");
-  PcPlan plan = plan_pc(chains, total_T, n_seqs, sms);
+  PcPlan plan = plan_pc(chains, total_T, n_seqs, Hv, sms);
   if (const char* env = getenv("GDN_TC_SLICE")) {
     const int v2 = atoi(env);
     if (v2 == 32 || v2 == 64 || v2 == 128) plan.dvp = v2;

@@ -1031,7 +1031,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         tc_fence_before();
         cbar();
         tc_fence_after();
-        if (tid == 0) {
+        if (tid == 0) {   // (a CTA's first package is published at once: chains are starting)
           bulk_store(pkg + kPkgA1, sm + L::kWm, 8192);
           bulk_store(pkg + kPkgA1 + 16384, sm + L::kWm + 8192, 8192);
           bulk_store(pkg + kPkgA1 + 8192, sm + L::kA1b, 8192);
@@ -1042,6 +1042,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           bulk_commit_group();
         }
         out_pending = b;
+        if (it == 0 && tid == 0) finish_out();
       }
       if (tid == 0) finish_out();
     }

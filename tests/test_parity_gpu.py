@@ -173,6 +173,16 @@ def test_prefill_workload_long_sampled_heads(T):
     check_prefill(workloads.inputs_for(w), w.tol_o, w.tol_state, heads=(0, 2) if T > 40000 else (0, 3))
 
 
+def test_prefill_many_short_sequences_many_rounds():
+    """300 sequences of 0..300 tokens x 8 value heads: far more sequence-heads than
+    chains run at once, so the tensor-core kernel works in many rounds whose
+    chains differ in length (numbers left unused in the package ring)."""
+    g = torch.Generator().manual_seed(4242)
+    lengths = [int(x) for x in torch.randint(0, 301, (300,), generator=g)]
+    x = workloads.prefill_inputs(lengths, Hqk=4, Hv=8, d=128, seed=4243, state_std=0.05)
+    check_prefill(x, 2e-2, 1e-2)
+
+
 def test_prefill_workload_varlen_sampled_heads():
     w = workloads.workload("varlen")
     check_prefill(workloads.inputs_for(w), w.tol_o, w.tol_state, heads=(0, 4))
