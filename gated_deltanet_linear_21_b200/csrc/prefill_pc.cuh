@@ -423,10 +423,12 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             __syncwarp();
             tc_fence_after();
             if (!early) issue_a2v(b);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma_bf16_warp(tmem + kColY, desc_kmajor(in + kPkgA1, kk, 16384), desc_mnmajor(sSb, kk, kRB, 128 * kRB),
-                            kIdY, 1u);
+            if (c > 0 || p.state_in != nullptr) {   // (a first chunk from a zero state has no A1 S^T;
+#pragma unroll                                        //  its package carries no A1)
+              for (int kk = 0; kk < 8; ++kk)
+                mma_bf16_warp(tmem + kColY, desc_kmajor(in + kPkgA1, kk, 16384), desc_mnmajor(sSb, kk, kRB, 128 * kRB),
+                              kIdY, 1u);
+            }
             mma_commit_warp(bar_mma);
             if (!mbar_wait(bar_u, ph_u)) { abort = true; break; }
             ph_u ^= 1;
@@ -625,6 +627,14 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           seq_bounds((int)(j / Hv), tb, te);
           c0 = tb + c * kC;
           len = min(kC, te - c0);
+          // the raw k, q tiles first: their latency covers the gates and the slot wait
+          const int hq = h / (Hv / Hqk);
+          uint8_t* kq = sm + L::kKQP + b * 32768;
+          mbar_expect_tx_warp(&bar_full[b], 4 * 8192);
+          tma_load_3d_warp(kq, &kmap, &bar_full[b], 0, hq, c0);
+          tma_load_3d_warp(kq + 16384, &kmap, &bar_full[b], 64, hq, c0);
+          tma_load_3d_warp(kq + 8192, &qmap, &bar_full[b], 0, hq, c0);
+          tma_load_3d_warp(kq + 16384 + 8192, &qmap, &bar_full[b], 64, hq, c0);
           float* qg = reinterpret_cast<float*>(qe + 16);
           float* qb = reinterpret_cast<float*>(qe + 80);
 #pragma unroll
@@ -641,19 +651,12 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           qe[1] = (uint32_t)s;
           qe[2] = (uint32_t)q;
           qe[3] = (uint32_t)len;
+          qe[4] = (uint32_t)c;
         }
         __syncwarp();
-        if (go) {
-          const int hq = h / (Hv / Hqk);
-          uint8_t* kq = sm + L::kKQP + b * 32768;
-          mbar_arrive_expect_tx_warp(&bar_full[b], 4 * 8192);
-          tma_load_3d_warp(kq, &kmap, &bar_full[b], 0, hq, c0);
-          tma_load_3d_warp(kq + 16384, &kmap, &bar_full[b], 64, hq, c0);
-          tma_load_3d_warp(kq + 8192, &qmap, &bar_full[b], 0, hq, c0);
-          tma_load_3d_warp(kq + 16384 + 8192, &qmap, &bar_full[b], 64, hq, c0);
-        } else if (lane == 0) {
-          mbar_arrive(&bar_full[b]);
-        }
+        // the arrival publishes the entry; the phase completes once the tiles are in too
+        // (an item that gave up after starting its tiles still lets them land first)
+        if (lane == 0) mbar_arrive(&bar_full[b]);
         return go;
       };
       for (int k = 0;; ++k) {
@@ -690,8 +693,10 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       float* Ad = reinterpret_cast<float*>(sm + L::kAd);
       float* scan = reinterpret_cast<float*>(&misc[2]);
 
-      // Thread 0: once the bulk copies of the previous package are complete, order
-      // them before the control warp's release and hand the item back.
+      // Thread 32 (warp 1, idle while the Gram product runs) owns the package's bulk
+      // copies: once those of the previous package are complete, it orders them
+      // before the publishing warp's release and hands the item back.
+      constexpr int kOutThread = 32;
       int out_pending = -1;
       auto finish_out = [&]() {
         if (out_pending < 0) return;
@@ -705,13 +710,16 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         const uint32_t* qe = reinterpret_cast<const uint32_t*>(sm + L::kQueue + b * L::kQueueBytes);
         // The previous package is published during this item's first stage, unless
         // this item is not here yet: its ring slot may wait for that package.
-        if (tid == 0 && out_pending >= 0 && !mbar_test_wait(&bar_full[b], (uint32_t)(it >> 1) & 1u)) finish_out();
+        if (tid == kOutThread && out_pending >= 0 && !mbar_test_wait(&bar_full[b], (uint32_t)(it >> 1) & 1u))
+          finish_out();
         {
           const bool w = mbar_wait(&bar_full[b], (uint32_t)(it >> 1) & 1u);
           if (!cbar_and(w)) { abort = true; break; }
         }
         if (qe[0] == 0) break;
         const int len = (int)qe[3];
+        // a chain's first chunk from a zero state never multiplies A1 (S = 0): skip -W, P W
+        const bool need_a1 = qe[4] != 0 || p.state_in != nullptr;
         uint8_t* pkg = pkgs + ((size_t)qe[2] * kRing + qe[1] % kRing) * kPkgStride;
         const uint32_t sKQ = sbase + L::kKQP + b * 32768;
 
@@ -721,7 +729,8 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           for (int kk = 0; kk < 8; ++kk)
             mma_bf16_warp(tmem + kColG, desc_kmajor(sKQ, kk, 16384), desc_kmajor(sKQ, kk, 16384), kIdG, kk > 0);
           mma_commit_warp(bar_mma);
-          if (lane == 0) finish_out();   // (before this item's vectors reuse the staging)
+        } else if (tid == kOutThread) {
+          finish_out();   // (before this item's vectors reuse the staging)
         }
         if (warp == 2 || warp == 3) {   // inclusive scan of g within each warp; the halves are joined below
           const int t = tid - 64, w2 = warp - 2;
@@ -785,6 +794,15 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           tmem_ld32(tmem + tlane + kColG + 32 * ch, gram);
           const int rr = r128 & 63;
           const float Gr = vGf[rr];
+          float ck[32];   // this thread's 32 columns of vCk, in 16-byte loads
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 t4 = reinterpret_cast<const float4*>(vCk + 32 * ch)[i];
+            ck[4 * i] = t4.x;
+            ck[4 * i + 1] = t4.y;
+            ck[4 * i + 2] = t4.z;
+            ck[4 * i + 3] = t4.w;
+          }
           float x[32];
           if (qd < 2) {
             const float fr = vB[rr] * vRk[rr] * (fast ? expf(Gr - gm) : 1.f);
@@ -792,13 +810,13 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
 #pragma unroll
               for (int q2 = 0; q2 < 32; ++q2) {
                 const int sidx = 32 * ch + q2;
-                x[q2] = (sidx < rr) ? fr * vCk[sidx] * gram[q2] : 0.f;
+                x[q2] = (sidx < rr) ? fr * ck[q2] * gram[q2] : 0.f;
               }
             } else {
 #pragma unroll
               for (int q2 = 0; q2 < 32; ++q2) {
                 const int sidx = 32 * ch + q2;
-                x[q2] = (sidx < rr) ? fr * vCk[sidx] * expf(Gr - vGf[sidx]) * gram[q2] : 0.f;
+                x[q2] = (sidx < rr) ? fr * ck[q2] * expf(Gr - vGf[sidx]) * gram[q2] : 0.f;
               }
             }
             const int blk = rr >> 4;
@@ -823,13 +841,13 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
 #pragma unroll
               for (int q2 = 0; q2 < 32; ++q2) {
                 const int sidx = 32 * ch + q2;
-                x[q2] = (sidx <= rr) ? fr * vCk[sidx] * gram[q2] : 0.f;
+                x[q2] = (sidx <= rr) ? fr * ck[q2] * gram[q2] : 0.f;
               }
             } else {
 #pragma unroll
               for (int q2 = 0; q2 < 32; ++q2) {
                 const int sidx = 32 * ch + q2;
-                x[q2] = (sidx <= rr) ? fr * vCk[sidx] * expf(Gr - vGf[sidx]) * gram[q2] : 0.f;
+                x[q2] = (sidx <= rr) ? fr * ck[q2] * expf(Gr - vGf[sidx]) * gram[q2] : 0.f;
               }
             }
 #pragma unroll
@@ -959,37 +977,41 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         // ---- -W = (-T_w) K_raw -> shared (operand of P W and A1 rows 0-63); the two
         //      column halves go to the two lane halves so that every thread has work ----
         const int dhalf = 64 * (lane >> 4) + 32 * ch;   // this thread's 32 columns of a d_k-wide row
-        if (warp == 0) {
+        if (need_a1) {
+          if (warp == 0) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_warp(tmem + kColW, desc_kmajor(sbase + L::kTw, kk, 0), desc_mnmajor(sKQ, kk, 128, 16384), kId64,
-                          kk > 0);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16_warp(tmem + kColW, desc_kmajor(sbase + L::kTw, kk, 0), desc_mnmajor(sKQ, kk, 128, 16384), kId64,
+                            kk > 0);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_warp(tmem + (16u << 16) + kColW, desc_kmajor(sbase + L::kTw, kk, 0),
-                          desc_mnmajor(sKQ + 16384, kk, 128, 16384), kId64, kk > 0);
-          mma_commit_warp(bar_mma);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16_warp(tmem + (16u << 16) + kColW, desc_kmajor(sbase + L::kTw, kk, 0),
+                            desc_mnmajor(sKQ + 16384, kk, 128, 16384), kId64, kk > 0);
+            mma_commit_warp(bar_mma);
+          }
+          if (!wait_mma()) { abort = true; break; }
+          {
+            float w[32];
+            tmem_ld32(tmem + tlane + kColW + 32 * ch, w);
+#pragma unroll
+            for (int c8 = 0; c8 < 4; ++c8)
+              st_shared_v4(sbase + L::kWm + sw128_off(r64, dhalf + 8 * c8, 8192), pack8_bf16(w + 8 * c8));
+          }
+          publish();
         }
-        if (!wait_mma()) { abort = true; break; }
-        {
-          float w[32];
-          tmem_ld32(tmem + tlane + kColW + 32 * ch, w);
-#pragma unroll
-          for (int c8 = 0; c8 < 4; ++c8)
-            st_shared_v4(sbase + L::kWm + sw128_off(r64, dhalf + 8 * c8, 8192), pack8_bf16(w + 8 * c8));
-        }
-        publish();
 
         // ---- -P W and P T_u -> A1 rows 64-127 = rho Q_raw - P W, A2 rows 64-127 = P T_u ----
         if (warp == 0) {
+          if (need_a1) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_warp(tmem + kColPW, desc_kmajor(sbase + L::kPm, kk, 0), desc_mnmajor(sbase + L::kWm, kk, 128, 8192),
-                          kId64, kk > 0);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16_warp(tmem + kColPW, desc_kmajor(sbase + L::kPm, kk, 0),
+                            desc_mnmajor(sbase + L::kWm, kk, 128, 8192), kId64, kk > 0);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_warp(tmem + (16u << 16) + kColPW, desc_kmajor(sbase + L::kPm, kk, 0),
-                          desc_mnmajor(sbase + L::kWm + 8192, kk, 128, 8192), kId64, kk > 0);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16_warp(tmem + (16u << 16) + kColPW, desc_kmajor(sbase + L::kPm, kk, 0),
+                            desc_mnmajor(sbase + L::kWm + 8192, kk, 128, 8192), kId64, kk > 0);
+          }
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_bf16_warp(tmem + kColPT, desc_kmajor(sbase + L::kPm, kk, 0), desc_mnmajor(sbase + L::kTu, kk, 128, 8192),
@@ -999,7 +1021,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         if (!wait_mma()) { abort = true; break; }
         {
           const float rho = vRho[r64];
-          {
+          if (need_a1) {
             float pw[32];
             tmem_ld32(tmem + tlane + kColPW + 32 * ch, pw);
 #pragma unroll
@@ -1031,20 +1053,22 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         tc_fence_before();
         cbar();
         tc_fence_after();
-        if (tid == 0) {   // (a CTA's first package is published at once: chains are starting)
-          bulk_store(pkg + kPkgA1, sm + L::kWm, 8192);
-          bulk_store(pkg + kPkgA1 + 16384, sm + L::kWm + 8192, 8192);
-          bulk_store(pkg + kPkgA1 + 8192, sm + L::kA1b, 8192);
-          bulk_store(pkg + kPkgA1 + 16384 + 8192, sm + L::kA1b + 8192, 8192);
+        if (tid == kOutThread) {   // (a CTA's first package is published at once: chains are starting)
+          if (need_a1) {
+            bulk_store(pkg + kPkgA1, sm + L::kWm, 8192);
+            bulk_store(pkg + kPkgA1 + 16384, sm + L::kWm + 8192, 8192);
+            bulk_store(pkg + kPkgA1 + 8192, sm + L::kA1b, 8192);
+            bulk_store(pkg + kPkgA1 + 16384 + 8192, sm + L::kA1b + 8192, 8192);
+          }
           bulk_store(pkg + kPkgA2, sm + L::kTu, 8192);
           bulk_store(pkg + kPkgA2 + 8192, sm + L::kA2b, 8192);
           bulk_store(pkg + kPkgUs, sm + L::kPv, kPkgCopy - kPkgUs);
           bulk_commit_group();
         }
         out_pending = b;
-        if (it == 0 && tid == 0) finish_out();
+        if (it == 0 && tid == kOutThread) finish_out();
       }
-      if (tid == 0) finish_out();
+      if (tid == kOutThread) finish_out();
     }
   }
 

@@ -263,6 +263,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx_warp(uint64_t* bar, uint32
       "r"(bytes)
       : "memory");
 }
+// Adds `bytes` to the barrier's expected transaction count without arriving
+// (warp-collective, one lane issues): copies may be started before the data
+// they travel with is written, and the arrival made afterwards.
+__device__ __forceinline__ void mbar_expect_tx_warp(uint64_t* bar, uint32_t bytes) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;\n\t}" ::"r"(smem_u32(bar)),
+      "r"(bytes)
+      : "memory");
+}
 __device__ __forceinline__ void tma_load_3d_warp(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
                                                  int z) {
   asm volatile(
