@@ -33,7 +33,7 @@ struct DecodeShape {
   static constexpr int kRowsPerSlot = 32 / kLanesPerRow;
   static constexpr int kSlots = 8 / kRowsPerSlot > 0 ? 8 / kRowsPerSlot : 1;  // 8 rows per warp
   static constexpr int kRowsPerWarp = kRowsPerSlot * kSlots;
-  static constexpr int kWarps = 4;
+  static constexpr int kWarps = 1;   // one-warp CTAs: the most independent loads in flight per SM
   static constexpr int kRowsPerCta = kRowsPerWarp * kWarps;
 };
 
@@ -57,21 +57,9 @@ decode_step_kernel(const TIO* __restrict__ q, const TIO* __restrict__ k,
   const int sub = lane % LPR;                // float4 index within the row
   const int slot_row = lane / LPR;           // row within a slot
 
-  // --- normalise q and k (every row group computes the same values) ---
-  const size_t qk_off = ((size_t)b * Hqk + hq) * DK + 4 * sub;
-  float4 kr = load4(k + qk_off);
-  float4 qr = load4(q + qk_off);
-  const float kinv = 1.0f / sqrtf(group_sum<LPR>(dot4(kr, kr)) + kNormEps);
-  const float qinv = scale / sqrtf(group_sum<LPR>(dot4(qr, qr)) + kNormEps);
-  const float4 kh = make_float4(kr.x * kinv, kr.y * kinv, kr.z * kinv, kr.w * kinv);
-  const float4 qh = make_float4(qr.x * qinv, qr.y * qinv, qr.z * qinv, qr.w * qinv);
-  const float kq = group_sum<LPR>(dot4(kh, qh));
-  const float alpha = expf(g[bh]);
-  const float bt = beta[bh];
-
+  // --- the state rows and v first: their latency covers the q, k normalisation ---
   const int row0 = blockIdx.y * Sh::kRowsPerCta + warp * Sh::kRowsPerWarp + slot_row;
   float4* S = reinterpret_cast<float4*>(state + (size_t)bh * dv * DK);
-
   float4 s[Sh::kSlots];
 #pragma unroll
   for (int j = 0; j < Sh::kSlots; ++j) {
@@ -84,6 +72,19 @@ decode_step_kernel(const TIO* __restrict__ q, const TIO* __restrict__ k,
     const int r = row0 + j * Sh::kRowsPerSlot;
     vv[j] = r < dv ? to_f32(v[(size_t)bh * dv + r]) : 0.f;
   }
+  const float alpha = expf(g[bh]);
+  const float bt = beta[bh];
+
+  // --- normalise q and k (every row group computes the same values) ---
+  const size_t qk_off = ((size_t)b * Hqk + hq) * DK + 4 * sub;
+  float4 kr = load4(k + qk_off);
+  float4 qr = load4(q + qk_off);
+  const float kinv = 1.0f / sqrtf(group_sum<LPR>(dot4(kr, kr)) + kNormEps);
+  const float qinv = scale / sqrtf(group_sum<LPR>(dot4(qr, qr)) + kNormEps);
+  const float4 kh = make_float4(kr.x * kinv, kr.y * kinv, kr.z * kinv, kr.w * kinv);
+  const float4 qh = make_float4(qr.x * qinv, qr.y * qinv, qr.z * qinv, qr.w * qinv);
+  const float kq = group_sum<LPR>(dot4(kh, qh));
+
 #pragma unroll
   for (int j = 0; j < Sh::kSlots; ++j) {
     const float a = group_sum<LPR>(dot4(s[j], kh));
