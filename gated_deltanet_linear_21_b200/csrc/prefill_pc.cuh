@@ -40,25 +40,32 @@
 //   chain CTAs each own one (sequence, value head, slice of DVP state rows) at a
 //              time and run only the state chain on the packages, k and v.
 //
-// Every CTA has eight compute warps and one control warp. The control warp
-// does what waits on other CTAs or on memory -- claiming items, polling and
-// publishing ring flags, issuing TMA and bulk copies -- a step ahead, and hands
-// work to the compute warps through mbarriers, which keeps those latencies off
-// the compute warps' critical path. Compute warps synchronise among themselves
-// with named barrier 1.
+// Every CTA has eight compute warps (0-7) and three with jobs of their own.
+// Warps 8 and 9 do what waits on other CTAs or on memory, a step ahead: in a
+// chain CTA warp 8 acquires ready flags and issues the copies of package, k
+// and v, and warp 9 hands ring slots back once a copy has landed; in a prep
+// CTA warp 8 claims items, fetches their gates and tiles and waits for ring
+// slots, and warp 9 publishes finished packages. In a chain CTA warp 10 issues
+// every tensor-core product and the O store, so the compute warps only run the
+// epilogues (U_s on warps 0, 1, 4, 5, O on 2, 3, 6, 7, then the state update);
+// in a prep CTA warp 0 issues the MMAs and warp 10 is idle. Handovers use
+// mbarriers with bounded waits; compute warps synchronise among themselves
+// with named barrier 1. (The register file is allocated per 128 threads, so
+// eleven warps cost no registers over nine.)
 //
 // Ring protocol. The chain CTAs work on the slice-chains in rounds; in round r
 // chain j = r P + q runs at position q < P (P chains per round). Each position
 // has a ring of R package slots and numbers its packages s = base_r + c, with
 // base_r the sum over earlier rounds of the longest chain's chunk count; slot
-// s mod R holds package s. The prep control warp waits until consumed[q][s mod R]
+// s mod R holds package s. The prep hand-over warp waits until consumed[q][s mod R]
 // >= slices * (s / R) (every slice read the previous occupant) before it hands
-// the item over, and once the compute warps have written the package it
-// publishes ready[q][s mod R] = s / R + 1 with release semantics; a chain control
-// warp waits for that value with acquire semantics, copies the package into
-// shared memory and then adds 1 to consumed[q][s mod R]. Numbers a shorter chain
-// leaves unused are counted as consumed by its chain CTAs at the end of the
-// round. Items are ordered by (round, chunk, chain), so a prep CTA never waits
+// the item over; the compute warps stage the package in shared memory and copy
+// it out with bulk copies, and once those are complete (and fenced) the
+// publishing warp sets ready[q][s mod R] = s / R + 1 with release semantics. A
+// chain's issuing warp waits for that value with acquire semantics and copies
+// the package into shared memory; its releasing warp then adds 1 to
+// consumed[q][s mod R]. Numbers a shorter chain leaves unused are counted as
+// consumed by its chain CTAs at the end of the round. Items are ordered by (round, chunk, chain), so a prep CTA never waits
 // on a chain that is not running, and the workspace holds P R packages however
 // many sequences there are. Every wait is bounded (~2 s): past it the CTA
 // records an error word and stops.

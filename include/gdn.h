@@ -107,6 +107,11 @@ size_t gdn_prefill_workspace_bytes(int n_seqs, int Hv, int dk, int dv, gdn_dtype
  * 74 at a time; larger problems return GDN_ERR_UNSUPPORTED (split them
  * across calls). It is one cooperative launch with one CTA on every SM of the
  * device: other work on the device runs before or after it, not beside it.
+ * How it splits the work (the width of the state slices and the number of
+ * CTAs that carry states) is chosen from the problem's shape; for experiments
+ * the environment variables GDN_TC_SLICE (32, 64 or 128 state rows) and
+ * GDN_PC_NC (number of state-carrying CTAs) override the choice. The result
+ * does not depend on either beyond rounding.
  * cu_seqlens is read on the device only; a cu_seqlens that breaks the rules
  * above is not detected on the host -- sequences with negative length are
  * treated as empty and tokens past total_T are never read.

@@ -183,6 +183,18 @@ def test_prefill_many_short_sequences_many_rounds():
     check_prefill(x, 2e-2, 1e-2)
 
 
+@pytest.mark.parametrize("dvp,nc", [(32, 0), (64, 0), (128, 0), (64, 6), (128, 3)])
+def test_prefill_every_slice_width_and_split(dvp, nc, monkeypatch):
+    """The tensor-core kernel with each state-slice width, and with so few
+    state-carrying CTAs that the chains run in several rounds; the result must
+    not change beyond rounding."""
+    monkeypatch.setenv("GDN_TC_SLICE", str(dvp))
+    if nc:
+        monkeypatch.setenv("GDN_PC_NC", str(nc))
+    x = workloads.prefill_inputs([300, 129, 64, 1], Hqk=4, Hv=8, d=128, seed=909 + dvp, state_std=0.05)
+    check_prefill(x, 2e-2, 1e-2)
+
+
 def test_prefill_workload_varlen_sampled_heads():
     w = workloads.workload("varlen")
     check_prefill(workloads.inputs_for(w), w.tol_o, w.tol_state, heads=(0, 4))
