@@ -278,9 +278,11 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     // chain: a buffer is free once the compute warps and the MMA warp are done with
     // it; U_s and O are staged by four warps each
     for (int i = 0; i < 8; ++i) {
-      const bool two = is_chain && (i == 2 || i == 3);
-      const bool four = is_chain && (i == 5 || i == 6);
-      mbar_init(&bar_full[i], two ? 2 : four ? 4 : 1);
+      uint32_t count = 1;
+      if (is_chain && (i == 2 || i == 3)) count = 9;   // free: the 8 compute warps and the MMA warp
+      if (is_chain && (i == 5 || i == 6)) count = 4;   // U_s / O staged: 4 warps each
+      if (is_chain && i == 7) count = 8;               // bf16 state written: the 8 compute warps
+      mbar_init(&bar_full[i], count);
     }
     fence_mbar_init();
     prefetch_tensormap(&qmap);
@@ -497,8 +499,8 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           };
           if (nch > 0) {
             store_state();
-            publish();
-            if (tid == 0) mbar_arrive(bar_s);
+            fence_async_smem();
+            warp_arrive(bar_s);
           }
 
           for (int c = 0; c < nch; ++c, ++gc) {
@@ -549,8 +551,12 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
               }
               store_state();
             }
-            publish();
-            if (tid == 0) {
+            // each warp tells the MMA warp its state rows are written and it is done with
+            // the buffer (no CTA-wide barrier here)
+            fence_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
               if (c + 1 < nch) mbar_arrive(bar_s);
               mbar_arrive(&bar_free[b]);
             }
