@@ -72,8 +72,10 @@ prefill_simt_kernel(const TIO* __restrict__ q, const TIO* __restrict__ k,
   const int tid = threadIdx.x, nthr = blockDim.x;
   const int lane = tid & 31, warp = tid >> 5, nwarp = nthr >> 5;
 
+  // a cu_seqlens that breaks its rules never makes a token outside [0, total_T) read
   long long t_begin = cu_seqlens[n], t_end = cu_seqlens[n + 1];
   if (t_end > total_T) t_end = total_T;
+  if (t_begin < 0) t_begin = 0;
   if (t_begin > t_end) t_begin = t_end;
 
   const size_t sbase = ((size_t)n * Hv + h) * (size_t)dv * dk + (size_t)i0 * dk;

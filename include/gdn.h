@@ -114,7 +114,7 @@ size_t gdn_prefill_workspace_bytes(int n_seqs, int Hv, int dk, int dv, gdn_dtype
  * does not depend on either beyond rounding.
  * cu_seqlens is read on the device only; a cu_seqlens that breaks the rules
  * above is not detected on the host -- sequences with negative length are
- * treated as empty and tokens past total_T are never read.
+ * treated as empty and tokens outside [0, total_T) are never read.
  */
 gdn_status gdn_prefill(const void *q, const void *k, const void *v,
                        const float *g, const float *beta,

@@ -173,6 +173,18 @@ def test_prefill_workload_long_sampled_heads(T):
     check_prefill(workloads.inputs_for(w), w.tol_o, w.tol_state, heads=(0, 2) if T > 40000 else (0, 3))
 
 
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_prefill_without_tokens_passes_the_states_through(dtype):
+    """Every sequence empty (total_T = 0): no output rows, state_out = state_in."""
+    x = workloads.prefill_inputs([0, 0, 0], Hqk=2, Hv=4, d=128, dtype=dtype, seed=31, state_std=0.05)
+    d = {kk: (vv.to(DEV) if isinstance(vv, torch.Tensor) else vv) for kk, vv in x.items()}
+    o, s = gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["state_in"], d["cu_seqlens"])
+    torch.cuda.synchronize()
+    gdn.device_error()
+    assert o.shape[0] == 0
+    assert torch.equal(s.cpu(), x["state_in"])
+
+
 def test_prefill_many_short_sequences_many_rounds():
     """300 sequences of 0..300 tokens x 8 value heads: far more sequence-heads than
     chains run at once, so the tensor-core kernel works in many rounds whose
