@@ -66,9 +66,9 @@ def prefill_bytes(T, Hqk, Hv, d, N, state_in):
     return b
 
 
-def decode_bytes(B, Hqk, Hv, d):
+def decode_bytes(B, Hqk, Hv, d, state_bytes=4):
     """Algorithmic HBM bytes of one decode step: state read + written, q, k, v, o, gates."""
-    return B * Hv * d * d * 4 * 2 + B * Hqk * d * 2 * 2 + B * Hv * d * 2 * 2 + B * Hv * 4 * 2
+    return B * Hv * d * d * state_bytes * 2 + B * Hqk * d * 2 * 2 + B * Hv * d * 2 * 2 + B * Hv * 4 * 2
 
 
 # the source files each kernel is built from (its traffic record is void once one changes)
@@ -252,7 +252,7 @@ def run_prefill_bench(gdn, w, steps, warmup, device, rank, sampler=None):
     return dict(ms=ms, tokens=T, bytes=one, copies=copies, graph=graph)
 
 
-def run_decode_bench(gdn, w, steps_timed, warmup, device, rank, sampler=None):
+def run_decode_bench(gdn, w, steps_timed, warmup, device, rank, sampler=None, state_dtype=torch.float32):
     stream = torch.cuda.current_stream()
     B, Hqk, Hv, d = w.batch, w.Hqk, w.Hv, w.d
     gen = torch.Generator(device=device).manual_seed(workloads.SEED_DECODE_STEP + 7919 * rank)
@@ -262,7 +262,7 @@ def run_decode_bench(gdn, w, steps_timed, warmup, device, rank, sampler=None):
     vs = torch.randn(n, B, Hv, d, generator=gen, device=device).to(torch.bfloat16)
     gs = torch.nn.functional.logsigmoid(torch.randn(n, B, Hv, generator=gen, device=device) + 3.0)
     bs = torch.sigmoid(torch.randn(n, B, Hv, generator=gen, device=device))
-    state = torch.randn(B, Hv, d, d, generator=gen, device=device) * w.state_std
+    state = (torch.randn(B, Hv, d, d, generator=gen, device=device) * w.state_std).to(state_dtype)
     o = torch.empty(B, Hv, d, dtype=torch.bfloat16, device=device)
 
     def run(a, b):
@@ -281,7 +281,7 @@ def run_decode_bench(gdn, w, steps_timed, warmup, device, rank, sampler=None):
             ms = timed(graph.replay, stream) / n
     else:
         ms = timed(graph.replay, stream) / n
-    return dict(ms=ms, bytes=decode_bytes(B, Hqk, Hv, d), steps=n)
+    return dict(ms=ms, bytes=decode_bytes(B, Hqk, Hv, d, state.element_size()), steps=n)
 
 
 def run_e2e(gdn, w, steps, device):
@@ -498,6 +498,13 @@ def main():
                           "config": workload_config(wd, None, world),
                           "roofline": roofline_hbm(rd["bytes"], rd["ms"], pk, pk_kind,
                                                    traffic=trd["bytes_per_launch"] if trd else None)}
+        # the same decode with the state stored in bf16 (gdn_decode_bf16_state)
+        rh = run_decode_bench(gdn, wd, wd.steps, args.warmup, device, rank, state_dtype=torch.bfloat16)
+        msh = max_over_ranks(rh["ms"])
+        line["decode_bf16_state"] = {"value": aggregate_rate(1, msh, world), "unit": "steps/s", "ms_per_step": msh,
+                                     "steps": rh["steps"], "gpu_launches": rh["steps"],
+                                     "config": dict(workload_config(wd, None, world), state="bf16 (fp32 arithmetic)"),
+                                     "roofline": roofline_hbm(rh["bytes"], rh["ms"], pk, pk_kind)}
         # one request at a time: B=1 decode, 1000 steps in one CUDA graph
         wb = workloads.Workload("decode_b1", 2, "decode", batch=1, steps=1000, Hqk=16, Hv=32,
                                 state_std=wd.state_std)

@@ -48,6 +48,7 @@ SIGNATURES = {
     "gdn_prefill": (_i, [_vp, _vp, _vp, _fp, _fp, _fp, _i32p, _i, _i64, _i, _i, _i, _i, _f, _i, _i,
                          _vp, _fp, _vp, _sz, _vp]),
     "gdn_decode": (_i, [_vp, _vp, _vp, _fp, _fp, _fp, _i, _i, _i, _i, _i, _f, _i, _vp, _vp]),
+    "gdn_decode_bf16_state": (_i, [_vp, _vp, _vp, _fp, _fp, _vp, _i, _i, _i, _i, _i, _f, _i, _vp, _vp]),
     "gdn_prefill_noalloc": (_i, [_vp, _vp, _vp, _fp, _fp, _fp, _i32p, _i, _i64, _i, _i, _i, _i, _f, _i, _i,
                                  _vp, _fp, _vp]),
     "gdn_device_error": (_i, [_vp]),
@@ -167,15 +168,20 @@ def prefill_noalloc(q, k, v, g, beta, state_in=None, cu_seqlens=None, *, scale=N
 
 def decode(q, k, v, g, beta, state, *, scale=None, o=None, stream=None):
     """One decode step: q, k [B, Hqk, dk]; v [B, Hv, dv]; g, beta [B, Hv];
-    state [B, Hv, dv, dk] fp32 updated in place. Returns o [B, Hv, dv]."""
+    state [B, Hv, dv, dk] updated in place -- fp32 (gdn_decode) or bf16
+    (gdn_decode_bf16_state: fp32 arithmetic, stored rounded to nearest even).
+    Returns o [B, Hv, dv]."""
     _dev(q, "q"); _dev(k, "k", q.dtype); _dev(v, "v", q.dtype)
     _dev(g, "g", torch.float32); _dev(beta, "beta", torch.float32)
-    _dev(state, "state", torch.float32)
+    _dev(state, "state")
+    if state.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError(f"state must be fp32 or bf16, got {state.dtype}")
     B, Hqk, dk = q.shape
     Hv, dv = v.shape[1], v.shape[2]
     if o is None:
         o = torch.empty(B, Hv, dv, dtype=q.dtype, device=q.device)
-    _check(lib().gdn_decode(
+    fn = lib().gdn_decode if state.dtype == torch.float32 else lib().gdn_decode_bf16_state
+    _check(fn(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), g.data_ptr(), beta.data_ptr(), state.data_ptr(),
         B, Hqk, Hv, dk, dv, float(scale or 0.0), _dtype_code(q), o.data_ptr(),
         _stream_handle(stream)))

@@ -17,19 +17,67 @@
 // which is the gated delta rule S' = alpha S (I - beta k^ k^^T) + beta v k^^T,
 // o = S' q^ with the product distributed so the row is read once.
 //
-// Layout: a row of DK fp32 is spread over DK/4 lanes as float4 (16-byte,
-// fully coalesced accesses); a warp holds NB row-slots in registers at once
-// so each lane keeps NB independent 16-byte loads in flight. Dot products
-// are reduced with butterfly shuffles inside the row's lane group.
+// Layout: a row of DK state values is spread over DK/4 (fp32) or DK/8 (bf16)
+// lanes as 16-byte chunks (fully coalesced accesses); a warp holds several
+// row-slots in registers at once so each lane keeps several independent
+// 16-byte loads in flight. Dot products are reduced with butterfly shuffles
+// inside the row's lane group. The state may be stored in fp32 or in bf16
+// (rounded to nearest even after each step); the arithmetic is fp32 either
+// way.
 #pragma once
 
 #include "common.cuh"
 
 namespace gdn {
 
-template <int DK>
+// 16 bytes of a state row: 4 fp32 or 8 bf16 values, moved with streaming
+// (evict-first) accesses since every state element is touched once per step.
+template <typename TS> struct StateChunk;
+template <> struct StateChunk<float> {
+  static constexpr int kElems = 4;
+  static __device__ __forceinline__ void load(const float* p, float* x) {
+    const float4 v = ld_stream(reinterpret_cast<const float4*>(p));
+    x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+  }
+  static __device__ __forceinline__ void store(float* p, const float* x) {
+    st_stream(reinterpret_cast<float4*>(p), make_float4(x[0], x[1], x[2], x[3]));
+  }
+};
+template <> struct StateChunk<__nv_bfloat16> {   // stored rounded to nearest even
+  static constexpr int kElems = 8;
+  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float* x) {
+    const uint4 v = __ldcs(reinterpret_cast<const uint4*>(p));
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(h[i]);
+      x[2 * i] = f.x;
+      x[2 * i + 1] = f.y;
+    }
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float* x) {
+    uint4 v;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+    __stcs(reinterpret_cast<uint4*>(p), v);
+  }
+};
+
+// E consecutive q/k elements as fp32 (E = 4 or 8)
+template <int E, typename T>
+__device__ __forceinline__ void load_vec(const T* p, float* x) {
+#pragma unroll
+  for (int i = 0; i < E; i += 4) {
+    const float4 v = load4(p + i);
+    x[i] = v.x; x[i + 1] = v.y; x[i + 2] = v.z; x[i + 3] = v.w;
+  }
+}
+
+template <int DK, typename TS>
 struct DecodeShape {
-  static constexpr int kLanesPerRow = DK / 4;
+  static constexpr int kElems = StateChunk<TS>::kElems;      // state elements per lane access
+  static constexpr int kLanesPerRow = DK / kElems;
   static constexpr int kRowsPerSlot = 32 / kLanesPerRow;
   static constexpr int kSlots = 8 / kRowsPerSlot > 0 ? 8 / kRowsPerSlot : 1;  // 8 rows per warp
   static constexpr int kRowsPerWarp = kRowsPerSlot * kSlots;
@@ -37,34 +85,36 @@ struct DecodeShape {
   static constexpr int kRowsPerCta = kRowsPerWarp * kWarps;
 };
 
-__device__ __forceinline__ float dot4(float4 a, float4 b) {
-  return a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w;
-}
-
 // grid: (B * Hv, ceil(dv / kRowsPerCta)); block: kWarps * 32
-template <typename TIO, int DK>
-__global__ void __launch_bounds__(DecodeShape<DK>::kWarps * 32)
+template <typename TIO, int DK, typename TS>
+__global__ void __launch_bounds__(DecodeShape<DK, TS>::kWarps * 32)
 decode_step_kernel(const TIO* __restrict__ q, const TIO* __restrict__ k,
                    const TIO* __restrict__ v, const float* __restrict__ g,
-                   const float* __restrict__ beta, float* __restrict__ state,
+                   const float* __restrict__ beta, TS* __restrict__ state,
                    int Hqk, int Hv, int dv, float scale, TIO* __restrict__ o) {
-  using Sh = DecodeShape<DK>;
+  using Sh = DecodeShape<DK, TS>;
+  constexpr int E = Sh::kElems;
   constexpr int LPR = Sh::kLanesPerRow;
   const int bh = blockIdx.x;                 // b * Hv + h
   const int b = bh / Hv, h = bh - b * Hv;
   const int hq = h / (Hv / Hqk);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int sub = lane % LPR;                // float4 index within the row
+  const int sub = lane % LPR;                // 16-byte chunk within the row
   const int slot_row = lane / LPR;           // row within a slot
 
   // --- the state rows and v first: their latency covers the q, k normalisation ---
   const int row0 = blockIdx.y * Sh::kRowsPerCta + warp * Sh::kRowsPerWarp + slot_row;
-  float4* S = reinterpret_cast<float4*>(state + (size_t)bh * dv * DK);
-  float4 s[Sh::kSlots];
+  TS* S = state + (size_t)bh * dv * DK;
+  float s[Sh::kSlots][E];
 #pragma unroll
   for (int j = 0; j < Sh::kSlots; ++j) {
     const int r = row0 + j * Sh::kRowsPerSlot;
-    s[j] = r < dv ? ld_stream(S + (size_t)r * LPR + sub) : make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r < dv) {
+      StateChunk<TS>::load(S + (size_t)r * DK + E * sub, s[j]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < E; ++e) s[j][e] = 0.f;
+    }
   }
   float vv[Sh::kSlots];
 #pragma unroll
@@ -76,28 +126,44 @@ decode_step_kernel(const TIO* __restrict__ q, const TIO* __restrict__ k,
   const float bt = beta[bh];
 
   // --- normalise q and k (every row group computes the same values) ---
-  const size_t qk_off = ((size_t)b * Hqk + hq) * DK + 4 * sub;
-  float4 kr = load4(k + qk_off);
-  float4 qr = load4(q + qk_off);
-  const float kinv = 1.0f / sqrtf(group_sum<LPR>(dot4(kr, kr)) + kNormEps);
-  const float qinv = scale / sqrtf(group_sum<LPR>(dot4(qr, qr)) + kNormEps);
-  const float4 kh = make_float4(kr.x * kinv, kr.y * kinv, kr.z * kinv, kr.w * kinv);
-  const float4 qh = make_float4(qr.x * qinv, qr.y * qinv, qr.z * qinv, qr.w * qinv);
-  const float kq = group_sum<LPR>(dot4(kh, qh));
+  const size_t qk_off = ((size_t)b * Hqk + hq) * DK + E * sub;
+  float kh[E], qh[E];
+  load_vec<E>(k + qk_off, kh);
+  load_vec<E>(q + qk_off, qh);
+  float kk = 0.f, qq = 0.f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    kk = fmaf(kh[e], kh[e], kk);
+    qq = fmaf(qh[e], qh[e], qq);
+  }
+  const float kinv = 1.0f / sqrtf(group_sum<LPR>(kk) + kNormEps);
+  const float qinv = scale / sqrtf(group_sum<LPR>(qq) + kNormEps);
+  float kq = 0.f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    kh[e] *= kinv;
+    qh[e] *= qinv;
+    kq = fmaf(kh[e], qh[e], kq);
+  }
+  kq = group_sum<LPR>(kq);
 
 #pragma unroll
   for (int j = 0; j < Sh::kSlots; ++j) {
-    const float a = group_sum<LPR>(dot4(s[j], kh));
-    const float bq = group_sum<LPR>(dot4(s[j], qh));
+    float a = 0.f, bq = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      a = fmaf(s[j][e], kh[e], a);
+      bq = fmaf(s[j][e], qh[e], bq);
+    }
+    a = group_sum<LPR>(a);
+    bq = group_sum<LPR>(bq);
     const int r = row0 + j * Sh::kRowsPerSlot;
     const float delta = bt * (vv[j] - alpha * a);
     if (r < dv) {
-      float4 ns;
-      ns.x = alpha * s[j].x + delta * kh.x;
-      ns.y = alpha * s[j].y + delta * kh.y;
-      ns.z = alpha * s[j].z + delta * kh.z;
-      ns.w = alpha * s[j].w + delta * kh.w;
-      st_stream(S + (size_t)r * LPR + sub, ns);
+      float ns[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) ns[e] = alpha * s[j][e] + delta * kh[e];
+      StateChunk<TS>::store(S + (size_t)r * DK + E * sub, ns);
       if (sub == 0) o[(size_t)bh * dv + r] = from_f32<TIO>(alpha * bq + delta * kq);
     }
   }

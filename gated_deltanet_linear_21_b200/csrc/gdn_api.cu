@@ -69,28 +69,53 @@ gdn_status launch_status(const char* what) {
 }
 
 // ---------------------------------------------------------------- decode ---
-template <typename TIO, int DK>
+template <typename TIO, int DK, typename TS>
 gdn_status launch_decode(const void* q, const void* k, const void* v, const float* g,
-                         const float* beta, float* state, int B, int Hqk, int Hv, int dv,
+                         const float* beta, TS* state, int B, int Hqk, int Hv, int dv,
                          float scale, void* o, cudaStream_t st) {
-  using Sh = gdn::DecodeShape<DK>;
+  using Sh = gdn::DecodeShape<DK, TS>;
   dim3 grid((unsigned)(B * Hv), (unsigned)((dv + Sh::kRowsPerCta - 1) / Sh::kRowsPerCta));
-  gdn::decode_step_kernel<TIO, DK><<<grid, Sh::kWarps * 32, 0, st>>>(
+  gdn::decode_step_kernel<TIO, DK, TS><<<grid, Sh::kWarps * 32, 0, st>>>(
       static_cast<const TIO*>(q), static_cast<const TIO*>(k), static_cast<const TIO*>(v), g, beta,
       state, Hqk, Hv, dv, scale, static_cast<TIO*>(o));
   return launch_status("gdn_decode");
 }
 
-template <typename TIO>
+template <typename TIO, typename TS>
 gdn_status dispatch_decode(const void* q, const void* k, const void* v, const float* g,
-                           const float* beta, float* state, int B, int Hqk, int Hv, int dk,
+                           const float* beta, TS* state, int B, int Hqk, int Hv, int dk,
                            int dv, float scale, void* o, cudaStream_t st) {
   switch (dk) {
-    case 16: return launch_decode<TIO, 16>(q, k, v, g, beta, state, B, Hqk, Hv, dv, scale, o, st);
-    case 32: return launch_decode<TIO, 32>(q, k, v, g, beta, state, B, Hqk, Hv, dv, scale, o, st);
-    case 64: return launch_decode<TIO, 64>(q, k, v, g, beta, state, B, Hqk, Hv, dv, scale, o, st);
-    default: return launch_decode<TIO, 128>(q, k, v, g, beta, state, B, Hqk, Hv, dv, scale, o, st);
+    case 16: return launch_decode<TIO, 16, TS>(q, k, v, g, beta, state, B, Hqk, Hv, dv, scale, o, st);
+    case 32: return launch_decode<TIO, 32, TS>(q, k, v, g, beta, state, B, Hqk, Hv, dv, scale, o, st);
+    case 64: return launch_decode<TIO, 64, TS>(q, k, v, g, beta, state, B, Hqk, Hv, dv, scale, o, st);
+    default: return launch_decode<TIO, 128, TS>(q, k, v, g, beta, state, B, Hqk, Hv, dv, scale, o, st);
   }
+}
+
+// Host checks shared by the decode entry points; GDN_OK when the call may proceed
+// (B == 0 is returned as done through *done).
+gdn_status check_decode(const char* fn, const void* q, const void* k, const void* v, const float* g,
+                        const float* beta, const void* state, int B, int Hqk, int Hv, int dk, int dv,
+                        gdn_dtype dtype, const void* o, bool* done) {
+  *done = false;
+  if (B < 0) return fail(GDN_ERR_INVALID_ARG, "%s: B=%d < 0", fn, B);
+  if (Hqk <= 0 || Hv <= 0 || Hv % Hqk != 0)
+    return fail(GDN_ERR_INVALID_ARG, "%s: Hv=%d must be a positive multiple of Hqk=%d", fn, Hv, Hqk);
+  if (!head_dim_ok(dk) || !head_dim_ok(dv))
+    return fail(GDN_ERR_UNSUPPORTED, "%s: dk=%d, dv=%d (supported: 16, 32, 64, 128)", fn, dk, dv);
+  if (dtype != GDN_BF16 && dtype != GDN_F32) return fail(GDN_ERR_INVALID_ARG, "%s: unknown dtype %d", fn, (int)dtype);
+  if ((int64_t)B * Hv > 0x7fffffff) return fail(GDN_ERR_INVALID_ARG, "%s: B*Hv too large", fn);
+  if (B == 0) {
+    *done = true;
+    return ok();
+  }
+  if (!q || !k || !v || !g || !beta || !state || !o)
+    return fail(GDN_ERR_INVALID_ARG, "%s: pointers must not be NULL", fn);
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(state))
+    return fail(GDN_ERR_INVALID_ARG, "%s: q, k, v, o and state must be 16-byte aligned", fn);
+  if (!aligned4(g) || !aligned4(beta)) return fail(GDN_ERR_INVALID_ARG, "%s: g and beta must be 4-byte aligned", fn);
+  return GDN_OK;
 }
 
 // --------------------------------------------------------------- prefill ---
@@ -351,26 +376,31 @@ gdn_status gdn_prefill(const void* q, const void* k, const void* v, const float*
 gdn_status gdn_decode(const void* q, const void* k, const void* v, const float* g,
                       const float* beta, float* state, int B, int Hqk, int Hv, int dk, int dv,
                       float scale, gdn_dtype dtype, void* o, void* stream) {
-  if (B < 0) return fail(GDN_ERR_INVALID_ARG, "gdn_decode: B=%d < 0", B);
-  if (Hqk <= 0 || Hv <= 0 || Hv % Hqk != 0)
-    return fail(GDN_ERR_INVALID_ARG, "gdn_decode: Hv=%d must be a positive multiple of Hqk=%d", Hv, Hqk);
-  if (!head_dim_ok(dk) || !head_dim_ok(dv))
-    return fail(GDN_ERR_UNSUPPORTED, "gdn_decode: dk=%d, dv=%d (supported: 16, 32, 64, 128)", dk, dv);
-  if (dtype != GDN_BF16 && dtype != GDN_F32)
-    return fail(GDN_ERR_INVALID_ARG, "gdn_decode: unknown dtype %d", (int)dtype);
-  if ((int64_t)B * Hv > 0x7fffffff) return fail(GDN_ERR_INVALID_ARG, "gdn_decode: B*Hv too large");
-  if (B == 0) return ok();
-  if (!q || !k || !v || !g || !beta || !state || !o)
-    return fail(GDN_ERR_INVALID_ARG, "gdn_decode: pointers must not be NULL");
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(state))
-    return fail(GDN_ERR_INVALID_ARG, "gdn_decode: q, k, v, o and state must be 16-byte aligned");
-  if (!aligned4(g) || !aligned4(beta))
-    return fail(GDN_ERR_INVALID_ARG, "gdn_decode: g and beta must be 4-byte aligned");
+  bool done = false;
+  if (gdn_status s = check_decode("gdn_decode", q, k, v, g, beta, state, B, Hqk, Hv, dk, dv, dtype, o, &done))
+    return s;
+  if (done) return ok();
   if (scale <= 0.f) scale = 1.0f / sqrtf((float)dk);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dtype == GDN_F32)
-    return dispatch_decode<float>(q, k, v, g, beta, state, B, Hqk, Hv, dk, dv, scale, o, st);
-  return dispatch_decode<__nv_bfloat16>(q, k, v, g, beta, state, B, Hqk, Hv, dk, dv, scale, o, st);
+    return dispatch_decode<float, float>(q, k, v, g, beta, state, B, Hqk, Hv, dk, dv, scale, o, st);
+  return dispatch_decode<__nv_bfloat16, float>(q, k, v, g, beta, state, B, Hqk, Hv, dk, dv, scale, o, st);
+}
+
+gdn_status gdn_decode_bf16_state(const void* q, const void* k, const void* v, const float* g,
+                                 const float* beta, void* state, int B, int Hqk, int Hv, int dk, int dv,
+                                 float scale, gdn_dtype dtype, void* o, void* stream) {
+  bool done = false;
+  if (gdn_status s =
+          check_decode("gdn_decode_bf16_state", q, k, v, g, beta, state, B, Hqk, Hv, dk, dv, dtype, o, &done))
+    return s;
+  if (done) return ok();
+  if (scale <= 0.f) scale = 1.0f / sqrtf((float)dk);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto* s16 = static_cast<__nv_bfloat16*>(state);
+  if (dtype == GDN_F32)
+    return dispatch_decode<float, __nv_bfloat16>(q, k, v, g, beta, s16, B, Hqk, Hv, dk, dv, scale, o, st);
+  return dispatch_decode<__nv_bfloat16, __nv_bfloat16>(q, k, v, g, beta, s16, B, Hqk, Hv, dk, dv, scale, o, st);
 }
 
 gdn_status gdn_wait_selftest(int max_wait_us, void* stream) {

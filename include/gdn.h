@@ -188,6 +188,22 @@ gdn_status gdn_decode(const void *q, const void *k, const void *v,
  */
 gdn_status gdn_wait_selftest(int max_wait_us, void *stream);
 
+/*
+ * gdn_decode with the state stored in bf16: the same step, computed in fp32,
+ * on a state [B, Hv, dv, dk] of bf16 values that is read, updated and written
+ * back rounded to nearest even -- the storage contract of "One level down:
+ * #004 the same compiler on Apple's chips", section "In short" (recurrence
+ * states in bf16, arithmetic in f32). It moves half the bytes of the fp32
+ * state per step; each step's rounding adds up to half a bf16 ulp per state
+ * element, so results drift from the fp32-state decode over many steps.
+ * o is computed from the updated state before it is rounded. Arguments,
+ * sizes and errors as gdn_decode; state is a DEVICE pointer to bf16 values.
+ */
+gdn_status gdn_decode_bf16_state(const void *q, const void *k, const void *v,
+                                 const float *g, const float *beta, void *state,
+                                 int B, int Hqk, int Hv, int dk, int dv,
+                                 float scale, gdn_dtype dtype, void *o, void *stream);
+
 /* Message describing the calling thread's most recent failure ("" if none). */
 const char *gdn_last_error(void);
 

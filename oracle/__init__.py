@@ -67,6 +67,10 @@ def _load():
                 ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                 ctypes.c_double, ctypes.c_double, ctypes.c_int, ctypes.c_int,
                 dp, ctypes.c_int]
+            lib.gdn_oracle_decode_ex.restype = ctypes.c_int
+            lib.gdn_oracle_decode_ex.argtypes = lib.gdn_oracle_decode.argtypes + [ctypes.c_int]
+            lib.gdn_oracle_round_bf16.restype = None
+            lib.gdn_oracle_round_bf16.argtypes = [dp, dp, ctypes.c_long]
             lib.gdn_oracle_max_threads.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -122,9 +126,19 @@ def prefill(q, k, v, g, beta, state_in, cu_seqlens, scale=None, eps=EPS,
     return o, s_out
 
 
-def decode(q, k, v, g, beta, state, scale=None, eps=EPS, heads=None, n_threads=None):
+def round_bf16(x) -> np.ndarray:
+    """fp64 values rounded to the nearest bfloat16 (ties to even) by way of the
+    nearest float, as the bf16-state decode stores them."""
+    x = _f64(x)
+    out = np.empty_like(x)
+    _load().gdn_oracle_round_bf16(_ptr(x), _ptr(out), x.size)
+    return out
+
+
+def decode(q, k, v, g, beta, state, scale=None, eps=EPS, heads=None, n_threads=None, state_bf16=False):
     """One fp64 decode step. ``state`` [B, Hv, dv, dk] (fp64 numpy) is updated in
-    place and also returned; returns (o [B, Hv, dv], state)."""
+    place and also returned; returns (o [B, Hv, dv], state). With ``state_bf16``
+    the updated state is stored rounded to bfloat16 (o is read before that)."""
     q, k, v, g, beta = (_f64(a) for a in (q, k, v, g, beta))
     if not (isinstance(state, np.ndarray) and state.dtype == np.float64
             and state.flags.c_contiguous):
@@ -137,9 +151,10 @@ def decode(q, k, v, g, beta, state, scale=None, eps=EPS, heads=None, n_threads=N
     o = np.full((B, Hv, dv), np.nan)
     if n_threads is None:
         n_threads = os.cpu_count() or 1
-    rc = _load().gdn_oracle_decode(
+    rc = _load().gdn_oracle_decode_ex(
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state),
-        B, Hqk, Hv, dk, dv, float(scale), float(eps), h_lo, h_hi, _ptr(o), int(n_threads))
+        B, Hqk, Hv, dk, dv, float(scale), float(eps), h_lo, h_hi, _ptr(o), int(n_threads),
+        1 if state_bf16 else 0)
     if rc != 0:
         raise ValueError("gdn_oracle_decode rejected its arguments")
     return o, state

@@ -158,11 +158,42 @@ int gdn_oracle_prefill(const double *q, const double *k, const double *v,
  * [B, Hv, dv, dk] is updated in place for value heads in [h_lo, h_hi);
  * o [B, Hv, dv] receives S_t q^_t for those heads.
  */
-int gdn_oracle_decode(const double *q, const double *k, const double *v,
-                      const double *g, const double *beta, double *state,
-                      int B, int Hqk, int Hv, int dk, int dv,
-                      double scale, double eps, int h_lo, int h_hi,
-                      double *o, int n_threads)
+/*
+ * x rounded to the nearest bfloat16, ties to even, by way of the nearest
+ * float (the value a computation carried in float would round): the 16 low
+ * bits of the float are dropped after adding half an ulp of the kept part
+ * plus its lowest bit. Infinities and NaN pass through.
+ */
+static double round_to_bf16(double x)
+{
+    float f = (float)x;
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7f800000u) == 0x7f800000u) return (double)f;
+    u += 0x7fffu + ((u >> 16) & 1u);
+    u &= 0xffff0000u;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* The rounding above over n values (exported so that tests can pin it). */
+void gdn_oracle_round_bf16(const double *x, double *out, long n)
+{
+    for (long i = 0; i < n; ++i) out[i] = round_to_bf16(x[i]);
+}
+
+/*
+ * One decode step (see gdn_oracle_decode). With round_state_bf16 the updated
+ * state is stored rounded to bfloat16 -- the storage contract of the Metal
+ * article ("One level down: #004 the same compiler on Apple's chips", section
+ * "In short": states kept in bf16, arithmetic in f32) -- after o has been
+ * read from the unrounded state.
+ */
+int gdn_oracle_decode_ex(const double *q, const double *k, const double *v,
+                         const double *g, const double *beta, double *state,
+                         int B, int Hqk, int Hv, int dk, int dv,
+                         double scale, double eps, int h_lo, int h_hi,
+                         double *o, int n_threads, int round_state_bf16)
 {
     if (B < 0 || Hqk <= 0 || Hv <= 0 || dk <= 0 || dv <= 0) return -1;
     if (Hv % Hqk != 0) return -1;
@@ -186,10 +217,24 @@ int gdn_oracle_decode(const double *q, const double *k, const double *v,
                             v + ((size_t)b * Hv + h) * dv,
                             g[(size_t)b * Hv + h], beta[(size_t)b * Hv + h],
                             scale, eps, o + ((size_t)b * Hv + h) * dv, work);
+            if (round_state_bf16) {
+                double *S = state + ((size_t)b * Hv + h) * (size_t)dv * dk;
+                for (size_t e = 0; e < (size_t)dv * dk; ++e) S[e] = round_to_bf16(S[e]);
+            }
         }
         free(work);
     }
     return 0;
+}
+
+int gdn_oracle_decode(const double *q, const double *k, const double *v,
+                      const double *g, const double *beta, double *state,
+                      int B, int Hqk, int Hv, int dk, int dv,
+                      double scale, double eps, int h_lo, int h_hi,
+                      double *o, int n_threads)
+{
+    return gdn_oracle_decode_ex(q, k, v, g, beta, state, B, Hqk, Hv, dk, dv, scale, eps, h_lo, h_hi, o,
+                                n_threads, 0);
 }
 
 /* Number of threads OpenMP would use by default (for reporting). */

@@ -263,3 +263,39 @@ def test_unmutated_copy_passes_pins(tmp_path, monkeypatch):
     subprocess.run(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-o",
                     str(tmp_path / "same.so"), str(tmp_path / "same.c"), "-lm"], check=True)
     assert _pins_pass(ctypes.CDLL(str(tmp_path / "same.so")), monkeypatch)
+
+
+# ------------------------------------------------- bf16-state decode variant ---
+
+def test_round_bf16_is_round_to_nearest_even_through_float():
+    """Pinned against torch's float -> bfloat16 conversion (round to nearest
+    even) on values of every magnitude, exact ties, subnormals and specials."""
+    import torch
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal(50000) * 10.0 ** rng.uniform(-40, 38, 50000)
+    ties = np.array([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -(1.0 + 2.0 ** -8), 2.0 ** -130, 0.0, -0.0])
+    x = np.concatenate([x, ties])
+    got = oracle.round_bf16(x)
+    ref = torch.tensor(x).to(torch.float32).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(got, ref)
+    # ties go to even: 1 + 2^-8 lies halfway between 1 and 1 + 2^-7 -> 1
+    assert got[-6] == 1.0 and got[-5] == 1.0 + 2.0 ** -6
+    sp = oracle.round_bf16(np.array([np.inf, -np.inf, np.nan]))
+    assert sp[0] == np.inf and sp[1] == -np.inf and np.isnan(sp[2])
+
+
+def test_bf16_state_decode_reads_o_before_rounding_and_stores_bf16():
+    B, Hqk, Hv, d = 2, 1, 2, 16
+    rng = np.random.default_rng(11)
+    state = oracle.round_bf16(rng.standard_normal((B, Hv, d, d)) * 0.1).reshape(B, Hv, d, d)
+    q, k, v = (rng.standard_normal((B, n, d)) for n in (Hqk, Hqk, Hv))
+    g = np.log(0.9) * np.ones((B, Hv))
+    beta = 0.5 * np.ones((B, Hv))
+    s64 = state.copy()
+    o64, s64 = oracle.decode(q, k, v, g, beta, s64)
+    s16 = state.copy()
+    o16, s16 = oracle.decode(q, k, v, g, beta, s16, state_bf16=True)
+    assert np.array_equal(o16, o64)                           # o from the unrounded state
+    assert np.array_equal(s16, oracle.round_bf16(s64).reshape(s64.shape))
+    assert np.array_equal(s16, oracle.round_bf16(s16).reshape(s16.shape))   # representable
+    assert not np.array_equal(s16, s64)

@@ -96,6 +96,51 @@ def test_decode_small(dtype, dk, dv):
     _gate("state", es, ms, 1e-2 if dtype == torch.bfloat16 else 1e-5)
 
 
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("dk,dv", [(16, 16), (64, 128), (128, 128), (128, 32)])
+def test_decode_bf16_state_small(dtype, dk, dv):
+    """gdn_decode_bf16_state against the oracle that stores the state rounded to
+    bf16 after each step (same storage contract); the arithmetic differs (fp32
+    vs fp64), so a rounding can land one bf16 ulp apart now and then."""
+    B, Hqk, Hv = 3, 2, 4
+    st = workloads.decode_state(B, Hv, dk, std=0.05, dv=dv).to(torch.bfloat16)
+    ref_state = st.double().numpy().copy()
+    sd = st.to(DEV)
+    for step in range(5):
+        x = workloads.decode_step_inputs(step, B, Hqk, Hv, dk, dtype, dv=dv)
+        o = gdn.decode(x["q"].to(DEV), x["k"].to(DEV), x["v"].to(DEV), x["g"].to(DEV), x["beta"].to(DEV), sd)
+        ro, ref_state = oracle.decode(x["q"], x["k"], x["v"], x["g"], x["beta"], ref_state, state_bf16=True)
+        eo, mo = _max_err(o, ro)
+        _gate("o", eo, mo, 2e-2)
+    es, ms = _max_err(sd, ref_state)
+    _gate("state", es, ms, 1e-2)
+
+
+def test_decode_bf16_state_workload_1000_steps_sampled_heads():
+    """The decode workload (64 sequences x 32 value heads, d=128, 1000 steps)
+    with a bf16 state, on value heads 0..3. Tolerances: one bf16 ulp of the
+    largest state value is about 1.2 * 2^-8 = 4.7e-3; rounding decisions that
+    fp32 and fp64 arithmetic take differently, once in a while, leave a few
+    such ulps after 1000 decaying steps: state <= 3e-2 (about 6 ulps),
+    o <= 3e-2."""
+    w = workloads.workload("decode")
+    heads = (0, 4)
+    st = workloads.decode_state(w.batch, w.Hv, w.d, std=w.state_std).to(torch.bfloat16)
+    ref = st.double().numpy().copy()
+    sd = st.to(DEV)
+    worst_o = 0.0
+    for step in range(w.steps):
+        x = workloads.decode_step_inputs(step, w.batch, w.Hqk, w.Hv, w.d)
+        o = gdn.decode(x["q"].to(DEV), x["k"].to(DEV), x["v"].to(DEV), x["g"].to(DEV), x["beta"].to(DEV), sd)
+        ro, ref = oracle.decode(x["q"], x["k"], x["v"], x["g"], x["beta"], ref, heads=heads, state_bf16=True)
+        eo, _ = _max_err(o, ro, (slice(None), slice(*heads)))
+        worst_o = max(worst_o, eo)
+    es, ms = _max_err(sd, ref, (slice(None), slice(*heads)))
+    print(f"bf16-state decode 1000 steps: worst o err {worst_o:.3e}, state err {es:.3e} (max|S| {ms:.3e})")
+    assert worst_o <= 3e-2
+    assert es <= 3e-2
+
+
 def test_decode_workload_1000_steps_sampled_heads():
     """64 sequences x 32 value heads, d=128, 1000 consecutive steps; o checked at
     every step and the state after the last one, on value heads 0..3."""
