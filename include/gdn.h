@@ -20,8 +20,8 @@
  * ("On descend d'un cran : #002 le même compilateur sur un GPU", section "Le
  * contrat numérique"; "One level down: #004", section "In short"). The
  * equation itself is not printed on the pages; the gated delta rule above is
- * the reading this library implements, and the fp32 state (rather than the
- * bf16 state the Metal article mentions) is this library's choice.
+ * the reading this library implements. States are fp32; gdn_decode_bf16_state
+ * also offers the Metal article's bf16 state storage for decode.
  *
  * Conventions shared by every entry point
  *   - All tensor arguments are DEVICE pointers (cudaMalloc'd or equivalent),
@@ -29,8 +29,8 @@
  *     The caller owns every buffer; the library never allocates, frees or
  *     synchronises (except gdn_device_error, which synchronises the stream).
  *   - dtype GDN_BF16: q, k, v, o are bf16 (o rounded to nearest even from
- *     fp32). GDN_F32: q, k, v, o are fp32. g, beta and the states are fp32
- *     in both cases.
+ *     fp32). GDN_F32: q, k, v, o are fp32. g and beta are fp32 in both
+ *     cases, and so are the states, except in gdn_decode_bf16_state.
  *   - Grouped heads: Hv must be a multiple of Hqk; value head h reads
  *     query/key head floor(h / (Hv / Hqk)) (contiguous groups).
  *   - g is the log-decay ln(alpha) (<= 0 in normal use); beta is used as given.
