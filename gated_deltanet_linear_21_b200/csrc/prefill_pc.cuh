@@ -50,7 +50,7 @@
 // epilogues (U_s on warps 0, 1, 4, 5, O on 2, 3, 6, 7, then the state update);
 // in a prep CTA warp 0 issues the MMAs and warp 10 is idle. Handovers use
 // mbarriers with bounded waits; compute warps synchronise among themselves
-// with named barrier 1. (The register file is allocated per 128 threads, so
+// with named barrier 1 (and the four O warps of a chain CTA with barrier 2). (The register file is allocated per 128 threads, so
 // eleven warps cost no registers over nine.)
 //
 // Ring protocol. The chain CTAs work on the slice-chains in rounds; in round r
@@ -128,8 +128,8 @@ constexpr uint32_t kColZ = 192;    // prep: N^2 E           M=64
 constexpr uint32_t kColW = 256;    // prep: -W, d_k 0-63 in lanes 0-15, 64-127 in lanes 16-31
 constexpr uint32_t kColPW = 320;   // prep: -P W, the same split
 constexpr uint32_t kColPT = 384;   // prep: P T_u           M=64, N=64 (lanes 0-15)
-constexpr uint32_t kColY = 0;      // chain: Y = [U ; O]    M=128, N=DVP
-constexpr uint32_t kColDS = 128;   // chain: dS^T           M=128, N=DVP
+constexpr uint32_t kColY = 0;      // chain: Y = [U ; O]    M=128, N=DVP, two buffers 128 columns apart
+constexpr uint32_t kColDS = 256;   // chain: dS^T           M=128, N=DVP
 
 template <int DVP>
 struct Smem {
@@ -242,7 +242,6 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
   uint64_t* bar_mma = bar_full + 4;
   uint64_t* bar_pub = bar_full + 5;                                  // [2] prep: publisher -> hand-over
   uint64_t* bar_u = bar_full + 5;      // chain: U_s staged (the 4 U warps)
-  uint64_t* bar_o = bar_full + 6;      // chain: O staged (the 4 O warps)
   uint64_t* bar_s = bar_full + 7;      // chain: the bf16 state copy is written
   uint32_t* misc = reinterpret_cast<uint32_t*>(sm + L::kMisc);     // [0] tmem, [2..5] scan
 
@@ -279,8 +278,8 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     // it; U_s and O are staged by four warps each
     for (int i = 0; i < 8; ++i) {
       uint32_t count = 1;
-      if (is_chain && (i == 2 || i == 3)) count = 9;   // free: the 8 compute warps and the MMA warp
-      if (is_chain && (i == 5 || i == 6)) count = 4;   // U_s / O staged: 4 warps each
+      if (is_chain && (i == 2 || i == 3)) count = 8;   // free: the 8 compute warps
+      if (is_chain && i == 5) count = 4;               // U_s staged: the 4 U warps
       if (is_chain && i == 7) count = 8;               // bf16 state written: the 8 compute warps
       mbar_init(&bar_full[i], count);
     }
@@ -404,19 +403,20 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       const uint32_t sSb = sbase + L::kSb;
       const uint32_t sUsb = sbase + L::kUsb;
       if (warp == kMmaWarp) {
-        // ---- MMA warp: per chunk Y = A2 V + A1 S^T (rows 0-63 U, rows 64-127 O), then
-        //      dS^T = K_raw^T U_s, the O store, and the next chunk's A2 V when its data
-        //      is in; it waits on the compute warps through mbarriers (bounded) ----
-        auto issue_a2v = [&](int b) {   // A2 V_raw of input buffer b, the first term of Y
+        // ---- MMA warp: per chunk Y = A2 V + A1 S^T (rows 0-63 U, rows 64-127 O) into
+        //      TMEM buffer gc & 1, then dS^T = K_raw^T U_s and, when the next chunk's
+        //      data is in, its A2 V into the other Y buffer; it waits on the compute
+        //      warps through mbarriers (bounded) ----
+        auto issue_a2v = [&](int b, uint32_t ycol) {   // A2 V_raw of input buffer b, the first term of Y
           const uint32_t in = sbase + L::kIn + b * L::kInBytes;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_warp(tmem + kColY, desc_kmajor(in + kPkgA2, kk, 0), desc_mnmajor(in + L::kInV, kk, kRB, 64 * kRB),
+            mma_bf16_warp(tmem + ycol, desc_kmajor(in + kPkgA2, kk, 0), desc_mnmajor(in + L::kInV, kk, kRB, 64 * kRB),
                           kIdY, kk > 0);
         };
         long gc = 0;
         bool early = false;
-        uint32_t ph_u = 0, ph_o = 0, ph_s = 0;
+        uint32_t ph_u = 0, ph_s = 0;
         for (long sc = blockIdx.x; sc < n_slice_chains && !abort; sc += NC) {
           long j;
           int h, i0, t_begin, t_end;
@@ -425,17 +425,16 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           for (int c = 0; c < nch; ++c, ++gc) {
             const int b = (int)(gc & 1);
             const uint32_t in = sbase + L::kIn + b * L::kInBytes;
-            const uint8_t* in_g = sm + L::kIn + b * L::kInBytes;
-            const bool o_tma = t_end - (t_begin + c * kC) >= kC;
+            const uint32_t ycol = kColY + 128u * (uint32_t)b;
             if (!mbar_wait(&bar_full[b], (uint32_t)(gc >> 1) & 1u) || !mbar_wait(bar_s, ph_s)) { abort = true; break; }
             ph_s ^= 1;
             __syncwarp();
             tc_fence_after();
-            if (!early) issue_a2v(b);
+            if (!early) issue_a2v(b, ycol);
             if (c > 0 || p.state_in != nullptr) {   // (a first chunk from a zero state has no A1 S^T;
 #pragma unroll                                        //  its package carries no A1)
               for (int kk = 0; kk < 8; ++kk)
-                mma_bf16_warp(tmem + kColY, desc_kmajor(in + kPkgA1, kk, 16384), desc_mnmajor(sSb, kk, kRB, 128 * kRB),
+                mma_bf16_warp(tmem + ycol, desc_kmajor(in + kPkgA1, kk, 16384), desc_mnmajor(sSb, kk, kRB, 128 * kRB),
                               kIdY, 1u);
             }
             mma_commit_warp(bar_mma);
@@ -448,30 +447,16 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
               mma_bf16_warp(tmem + kColDS, desc_mnmajor(in + L::kInK, kk, 128, 8192),
                             desc_mnmajor(sUsb, kk, kRB, 64 * kRB), kIdDS, kk > 0);
             mma_commit_warp(bar_mma);
-            if (!mbar_wait(bar_o, ph_o)) { abort = true; break; }
-            ph_o ^= 1;
-            __syncwarp();
-            tc_fence_after();
-            if (lane == 0 && o_tma) {   // O of a whole chunk goes out from the v tile's place
-#pragma unroll
-              for (int vb = 0; vb < L::kBlocks; ++vb)
-                tma_store_3d(&omap, in_g + L::kInV + vb * 64 * kRB, i0 + vb * L::kBlk, h, t_begin + c * kC);
-              bulk_commit_group();
-            }
-            __syncwarp();
+            // the other Y buffer was last read in chunk gc - 1, whose epilogues all ended
+            // before the compute warps' state update of that chunk (and so before bar_u)
             early = false;
             if (c + 1 < nch) {
               const bool nxt = mbar_test_wait(&bar_full[b ^ 1], (uint32_t)((gc + 1) >> 1) & 1u);
               if (__shfl_sync(0xffffffffu, nxt ? 1 : 0, 0)) {
-                issue_a2v(b ^ 1);
+                issue_a2v(b ^ 1, kColY + 128u * (uint32_t)(b ^ 1));
                 early = true;
               }
             }
-            if (lane == 0) {
-              bulk_wait_read_all();   // the O tile has left the buffer
-              mbar_arrive(&bar_free[b]);
-            }
-            __syncwarp();
           }
         }
       } else {
@@ -517,7 +502,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
 #pragma unroll
               for (int pp = 0; pp < kHalf / kPart; ++pp) {
                 float yv[kPart];
-                tmem_ld<kPart>(tmem + tlane + kColY + ch * kHalf + pp * kPart, yv);
+                tmem_ld<kPart>(tmem + tlane + kColY + 128u * (uint32_t)b + ch * kHalf + pp * kPart, yv);
                 if (qd < 2) {   // U_s = diag(us) U -> shared memory (bf16) for dS
 #pragma unroll
                   for (int q2 = 0; q2 < kPart; ++q2) yv[q2] *= us;
@@ -538,7 +523,17 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             }
             fence_async_smem();
             tc_fence_before();
-            warp_arrive(qd < 2 ? bar_u : bar_o);
+            if (qd < 2) {
+              warp_arrive(bar_u);
+            } else if (o_tma) {   // the O warps meet, then thread 64 stores the O tile
+              named_bar_sync(2, 128);
+              if (tid == 64) {
+#pragma unroll
+                for (int vb = 0; vb < L::kBlocks; ++vb)
+                  tma_store_3d(&omap, in_g + L::kInV + vb * 64 * kRB, i0 + vb * L::kBlk, h, t_begin + c * kC);
+                bulk_commit_group();
+              }
+            }
             if (!wait_mma()) { abort = true; break; }   // dS
             {
               const float gL = *reinterpret_cast<const float*>(in_g + kPkgGL);
@@ -555,6 +550,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             // the buffer (no CTA-wide barrier here)
             fence_async_smem();
             tc_fence_before();
+            if (tid == 64) bulk_wait_read_all();   // the O tile has left the buffer
             __syncwarp();
             if (lane == 0) {
               if (c + 1 < nch) mbar_arrive(bar_s);
