@@ -46,8 +46,8 @@
 // and v, and warp 9 hands ring slots back once a copy has landed; in a prep
 // CTA warp 8 claims items, fetches their gates and tiles and waits for ring
 // slots, and warp 9 publishes finished packages. In a chain CTA warp 10 issues
-// every tensor-core product and the O store, so the compute warps only run the
-// epilogues (U_s on warps 0, 1, 4, 5, O on 2, 3, 6, 7, then the state update);
+// every tensor-core product, so the compute warps only run the epilogues (U_s
+// on warps 0, 1, 4, 5, O on 2, 3, 6, 7, which also store O; then the state);
 // in a prep CTA warp 0 issues the MMAs and warp 10 is idle. Handovers use
 // mbarriers with bounded waits; compute warps synchronise among themselves
 // with named barrier 1 (and the four O warps of a chain CTA with barrier 2). (The register file is allocated per 128 threads, so
@@ -90,7 +90,7 @@ constexpr int kCompute = 256;        // compute threads (warps 0-7)
 constexpr int kThreads = 352;        // and three warps with their own jobs:
 constexpr int kCtlWarp = 8;          // chain: issues the copies; prep: claims and hands over items
 constexpr int kRelWarp = 9;          // chain: hands ring slots back; prep: publishes packages
-constexpr int kMmaWarp = 10;         // chain: issues the tensor-core work and the O store
+constexpr int kMmaWarp = 10;         // chain: issues the tensor-core work
 constexpr uint32_t kTmemCols = 512;
 constexpr int kRing = 12;            // package slots per ring position
 constexpr int kMaxRounds = 1024;
