@@ -275,10 +275,12 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
 
   if (tid == 0) {
     // chain: a buffer is free once the compute warps and the MMA warp are done with
-    // it; U_s and O are staged by four warps each
+    // it and the releasing warp has seen its copy land (so that the releasing warp,
+    // which waits by parity, never falls a phase behind); U_s and O are staged by
+    // four warps each
     for (int i = 0; i < 8; ++i) {
       uint32_t count = 1;
-      if (is_chain && (i == 2 || i == 3)) count = 8;   // free: the 8 compute warps
+      if (is_chain && (i == 2 || i == 3)) count = 9;   // free: the 8 compute warps + the releasing warp
       if (is_chain && i == 5) count = 4;               // U_s staged: the 4 U warps
       if (is_chain && i == 7) count = 8;               // bf16 state written: the 8 compute warps
       mbar_init(&bar_full[i], count);
@@ -388,9 +390,12 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         const int nch = (t_end - t_begin + kC - 1) / kC;
         const int maxc = round_maxc(j, q);
         for (int c = 0; c < nch; ++c, ++gc) {
-          // (if this warp is two phases behind, the wait ends with a later copy: only later)
           if (!mbar_wait(&bar_full[gc & 1], (uint32_t)(gc >> 1) & 1u)) { abort = true; break; }
-          if (lane == 0) red_add_release_gpu(&cns[(base + c) % kRing], 1u);
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&bar_free[gc & 1]);   // (the buffer is not refilled before this)
+            red_add_release_gpu(&cns[(base + c) % kRing], 1u);
+          }
         }
         if (abort) break;
         if (lane == 0)

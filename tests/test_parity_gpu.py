@@ -252,6 +252,17 @@ def test_prefill_every_slice_width_and_split(dvp, nc, monkeypatch):
     check_prefill(x, 2e-2, 1e-2)
 
 
+@pytest.mark.parametrize("dvp,nc", [(32, 4), (64, 2), (64, 4), (128, 2)])
+def test_prefill_long_chains_in_several_rounds(dvp, nc, monkeypatch):
+    """Chains far longer than the package ring (2500 tokens: 40 chunks, the ring
+    wraps three times per chain) run in two to four rounds: every ring slot is
+    reused many times within a round and across the round boundary."""
+    monkeypatch.setenv("GDN_TC_SLICE", str(dvp))
+    monkeypatch.setenv("GDN_PC_NC", str(nc))
+    x = workloads.prefill_inputs([2500], Hqk=2, Hv=4, d=128, seed=5150 + dvp + nc, state_std=0.05)
+    check_prefill(x, 2e-2, 1e-2)
+
+
 def test_prefill_workload_varlen_sampled_heads():
     w = workloads.workload("varlen")
     check_prefill(workloads.inputs_for(w), w.tol_o, w.tol_state, heads=(0, 4))
