@@ -79,7 +79,10 @@ struct DecodeShape {
   static constexpr int kElems = StateChunk<TS>::kElems;      // state elements per lane access
   static constexpr int kLanesPerRow = DK / kElems;
   static constexpr int kRowsPerSlot = 32 / kLanesPerRow;
-  static constexpr int kSlots = 8 / kRowsPerSlot > 0 ? 8 / kRowsPerSlot : 1;  // 8 rows per warp
+  // 8 fp32 rows or 16 bf16 rows per warp: at d_k = 128 every lane keeps 8 independent
+  // 16-byte loads in flight whatever the state's type
+  static constexpr int kRowsTarget = 8 * (int)(sizeof(float) / sizeof(TS));
+  static constexpr int kSlots = kRowsTarget / kRowsPerSlot > 0 ? kRowsTarget / kRowsPerSlot : 1;
   static constexpr int kRowsPerWarp = kRowsPerSlot * kSlots;
   static constexpr int kWarps = 1;   // one-warp CTAs: the most independent loads in flight per SM
   static constexpr int kRowsPerCta = kRowsPerWarp * kWarps;

@@ -106,7 +106,7 @@ constexpr uint32_t kPkgStride = 50176;
 
 // ---- workspace layout ----
 struct Workspace {
-  static constexpr size_t kCounter = 0;      // uint32 item counter
+  static constexpr size_t kCounter = 0;      // uint32 counter of the items after the first one per prep CTA
   static constexpr size_t kFlags = 256;      // ready[positions][R], then consumed[positions][R]
   __host__ __device__ static constexpr size_t flags_bytes(long positions) {
     return (size_t)positions * kRing * 2 * sizeof(uint32_t);
@@ -609,8 +609,12 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         int v = 0, c = 0, q = 0, s = 0;
         long j = 0;
         if (lane == 0) {
+          // a CTA's first item is fixed (items [0, prep CTAs), one each: no contended
+          // atomic on the way to the first packages); the counter numbers the rest
+          bool first = k == 0;
           while (true) {
-            const int item = (int)atomicAdd(counter, 1u);
+            const int item = first ? (int)blockIdx.x - NC : ((int)gridDim.x - NC) + (int)atomicAdd(counter, 1u);
+            first = false;
             if (item >= total_items) break;
             int r = 0, hi = n_rounds - 1;   // the round holding the item
             while (r < hi) {
@@ -656,7 +660,8 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             qg[e] = e < len ? p.g[(size_t)(c0 + e) * Hv + h] : 0.f;
             qb[e] = e < len ? p.beta[(size_t)(c0 + e) * Hv + h] : 0.f;
           }
-          if (lane == 0) ok = wait_flag_geq(&consumed[q * kRing + s % kRing], (uint32_t)(kSlices * (s / kRing)));
+          // (numbers below kRing have no previous occupant to wait for)
+          if (lane == 0 && s >= kRing) ok = wait_flag_geq(&consumed[q * kRing + s % kRing], (uint32_t)(kSlices * (s / kRing)));
           ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         }
         const bool go = v && ok;
