@@ -295,32 +295,64 @@ def run_decode_bench(gdn, w, steps_timed, warmup, device, rank, sampler=None, st
 
 
 def run_e2e(gdn, w, steps, device):
-    """Same prefill through the public API with inputs in pinned host memory:
-    H2D of q, k, v, g, beta, the call, and D2H of o and the final states."""
-    stream = torch.cuda.current_stream()
+    """Same prefill through the public API with inputs in pinned host memory: every
+    step copies q, k, v, g, beta (and the states) up, calls gdn.prefill and copies o
+    and the final states down. Steps are pipelined the way a serving loop runs them:
+    step i+1's inputs go up on one copy stream while step i computes and step i-1's
+    results come down on another (PCIe carries both directions at once), over two
+    sets of device buffers ordered by events. The timed region, on the launching
+    stream, holds every step's copies and calls."""
+    main = torch.cuda.current_stream()
     x = workloads.inputs_for(w) if w.total_tokens <= 8192 else None
     if x is None:
         x = {kk: (vv.cpu() if isinstance(vv, torch.Tensor) else vv)
              for kk, vv in device_prefill_inputs(w.lengths, w.Hqk, w.Hv, w.d, 11, device).items()}
     host = {kk: vv.pin_memory() for kk, vv in x.items() if isinstance(vv, torch.Tensor)}
-    dev = {kk: torch.empty_like(vv, device=device) for kk, vv in host.items()}
     T, N = w.total_tokens, len(w.lengths)
     o_h = torch.empty(T, w.Hv, w.d, dtype=torch.bfloat16).pin_memory()
     s_h = torch.empty(N, w.Hv, w.d, w.d).pin_memory()
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = o_h.numel() * o_h.element_size() + s_h.numel() * s_h.element_size()
+    sets = [({kk: torch.empty_like(vv, device=device) for kk, vv in host.items()},
+             torch.empty(T, w.Hv, w.d, dtype=torch.bfloat16, device=device),
+             torch.empty(N, w.Hv, w.d, w.d, dtype=torch.float32, device=device)) for _ in range(2)]
+    ws = torch.empty(max(1, gdn.prefill_workspace_bytes(N, w.Hv, w.d, w.d)), dtype=torch.uint8, device=device)
+    up, cmp, down = (torch.cuda.Stream(device=device) for _ in range(3))
+    ev_up, ev_cmp, ev_down = ([torch.cuda.Event() for _ in range(2)] for _ in range(3))
 
-    def step():
-        for kk in host:
-            dev[kk].copy_(host[kk], non_blocking=True)
-        o, s = gdn.prefill(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], dev.get("state_in"),
-                           dev["cu_seqlens"])
-        o_h.copy_(o, non_blocking=True)
-        s_h.copy_(s, non_blocking=True)
+    def step(i):
+        b = i & 1
+        dev, o_d, s_d = sets[b]
+        up.wait_event(ev_cmp[b])     # the call two steps back has read these inputs
+        with torch.cuda.stream(up):
+            for kk in host:
+                dev[kk].copy_(host[kk], non_blocking=True)
+        ev_up[b].record(up)
+        cmp.wait_event(ev_up[b])
+        cmp.wait_event(ev_down[b])   # the results two steps back have left these outputs
+        gdn.prefill(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], dev.get("state_in"),
+                    dev["cu_seqlens"], o=o_d, state_out=s_d, workspace=ws, stream=cmp)
+        ev_cmp[b].record(cmp)
+        down.wait_event(ev_cmp[b])
+        with torch.cuda.stream(down):
+            o_h.copy_(o_d, non_blocking=True)
+            s_h.copy_(s_d, non_blocking=True)
+        ev_down[b].record(down)
 
-    for _ in range(2):
-        step()
-    ms = timed(lambda: [step() for _ in range(steps)], stream) / steps
+    def run(n):
+        start = torch.cuda.Event()
+        start.record(main)
+        for st in (up, cmp, down):
+            st.wait_event(start)
+        for i in range(n):
+            step(i)
+        for st in (up, cmp, down):
+            e = torch.cuda.Event()
+            e.record(st)
+            main.wait_event(e)
+
+    run(2)
+    ms = timed(lambda: run(steps), main) / steps
     return dict(ms=ms, h2d=h2d, d2h=d2h, tokens=T)
 
 

@@ -263,6 +263,30 @@ def test_prefill_long_chains_in_several_rounds(dvp, nc, monkeypatch):
     check_prefill(x, 2e-2, 1e-2)
 
 
+def test_prefill_on_a_side_stream_into_caller_buffers():
+    """The call enqueues on the stream it is given and writes caller-owned o,
+    state_out and workspace, as a pipelined loop (copies on other streams) uses it."""
+    x = workloads.prefill_inputs([200, 77], Hqk=2, Hv=4, d=128, seed=777, state_std=0.05)
+    d = {kk: (vv.to(DEV) if isinstance(vv, torch.Tensor) else vv) for kk, vv in x.items()}
+    T, Hv, dv = d["v"].shape
+    N = d["cu_seqlens"].numel() - 1
+    side = torch.cuda.Stream()
+    o = torch.full((T, Hv, dv), float("nan"), dtype=torch.bfloat16, device=DEV)
+    s_out = torch.full((N, Hv, dv, 128), float("nan"), dtype=torch.float32, device=DEV)
+    ws = torch.empty(gdn.prefill_workspace_bytes(N, Hv, 128, dv), dtype=torch.uint8, device=DEV)
+    side.wait_stream(torch.cuda.current_stream())
+    ro_, rs_ = gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["state_in"], d["cu_seqlens"],
+                           o=o, state_out=s_out, workspace=ws, stream=side)
+    assert ro_ is o and rs_ is s_out
+    side.synchronize()
+    gdn.device_error(stream=side)
+    ro, rs = oracle.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], x["state_in"], x["cu_seqlens"])
+    eo, mo = _max_err(o, ro, None)
+    es, ms = _max_err(s_out, rs, None)
+    _gate("o", eo, mo, 2e-2)
+    _gate("state", es, ms, 1e-2)
+
+
 def test_prefill_workload_varlen_sampled_heads():
     w = workloads.workload("varlen")
     check_prefill(workloads.inputs_for(w), w.tol_o, w.tol_state, heads=(0, 4))
