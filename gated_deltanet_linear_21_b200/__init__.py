@@ -16,7 +16,8 @@ import threading
 
 import torch
 
-__all__ = ["prefill", "prefill_noalloc", "decode", "prefill_workspace_bytes", "device_error", "wait_selftest",
+__all__ = ["prefill", "prefill_noalloc", "decode", "prefill_workspace_bytes", "prefill_plan", "device_error",
+           "wait_selftest",
            "GdnError",
            "lib", "library_path", "GDN_BF16", "GDN_F32"]
 
@@ -53,6 +54,7 @@ SIGNATURES = {
                                  _vp, _fp, _vp]),
     "gdn_device_error": (_i, [_vp]),
     "gdn_wait_selftest": (_i, [_i, _vp]),
+    "gdn_prefill_plan": (_i, [_i, _i64, _i, _i, _i, _i, _i, _vp, _vp, _vp]),
 }
 
 
@@ -104,6 +106,17 @@ def _stream_handle(stream) -> int:
 def prefill_workspace_bytes(n_seqs, Hv, dk, dv, dtype=torch.bfloat16) -> int:
     code = GDN_BF16 if dtype == torch.bfloat16 else GDN_F32
     return int(lib().gdn_prefill_workspace_bytes(n_seqs, Hv, dk, dv, code))
+
+
+def prefill_plan(n_seqs, total_T, Hv, dk=128, dv=128, dtype=torch.bfloat16, sm_count=0):
+    """(dvp, n_chain_ctas, rounds): the launch plan the tensor-core prefill would
+    use for this problem (the GDN_TC_SLICE / GDN_PC_NC overrides included);
+    host only. sm_count=0 asks the current device."""
+    code = GDN_BF16 if dtype == torch.bfloat16 else GDN_F32
+    out = [ctypes.c_int(0) for _ in range(3)]
+    _check(lib().gdn_prefill_plan(int(n_seqs), int(total_T), int(Hv), int(dk), int(dv), code, int(sm_count),
+                                  *[ctypes.byref(x) for x in out]))
+    return tuple(x.value for x in out)
 
 
 def prefill(q, k, v, g, beta, state_in=None, cu_seqlens=None, *, scale=None, chunk=0,

@@ -269,12 +269,14 @@ PcPlan plan_pc(long chains, int64_t total_T, int n_seqs, int Hv, int sms) {
   return best;
 }
 
-gdn_status launch_prefill_pc(const void* q, const void* k, const void* v, const float* g, const float* beta,
-                             const float* state_in, const int32_t* cu, int n_seqs, int64_t total_T, int Hqk,
-                             int Hv, float scale, void* o, float* state_out, void* ws, cudaStream_t st) {
-  const long chains = (long)n_seqs * Hv;
-  const int sms = sm_count();
-  if (sms < 16) return fail(GDN_ERR_CUDA, "gdn_prefill: cannot query the multiprocessor count");
+// The plan a launch uses: the model's choice, then the GDN_TC_SLICE / GDN_PC_NC
+// overrides, clamped so that no position is without a chain, a chain's slices
+// stay in one round and the package ring's positions suffice.
+struct PcLaunchPlan {
+  int dvp;
+  long nc, rounds;
+};
+PcLaunchPlan resolve_pc(long chains, int64_t total_T, int n_seqs, int Hv, int sms) {
   PcPlan plan = plan_pc(chains, total_T, n_seqs, Hv, sms);
   if (const char* env = getenv("GDN_TC_SLICE")) {
     const int v2 = atoi(env);
@@ -287,8 +289,19 @@ gdn_status launch_prefill_pc(const void* q, const void* k, const void* v, const 
   nc = std::min(nc, (long)gdn::pc::kMaxPositions * slices);
   nc -= nc % slices;
   if (nc < slices) nc = slices;
-  const long rounds = (chains * slices + nc - 1) / nc;
-  if (rounds > gdn::pc::kMaxRounds)
+  return {dvp, nc, (chains * slices + nc - 1) / nc};
+}
+
+gdn_status launch_prefill_pc(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                             const float* state_in, const int32_t* cu, int n_seqs, int64_t total_T, int Hqk,
+                             int Hv, float scale, void* o, float* state_out, void* ws, cudaStream_t st) {
+  const long chains = (long)n_seqs * Hv;
+  const int sms = sm_count();
+  if (sms < 16) return fail(GDN_ERR_CUDA, "gdn_prefill: cannot query the multiprocessor count");
+  const PcLaunchPlan lp = resolve_pc(chains, total_T, n_seqs, Hv, sms);
+  const int dvp = lp.dvp, slices = 128 / dvp;
+  const long nc = lp.nc;
+  if (lp.rounds > gdn::pc::kMaxRounds)
     return fail(GDN_ERR_UNSUPPORTED, "gdn_prefill: %ld sequence-heads is more than this kernel schedules", chains);
   CUtensorMap qm, km, vm, om;
   if (!make_map(&qm, q, 128, Hqk, (int)total_T, 64) || !make_map(&km, k, 128, Hqk, (int)total_T, 64) ||
@@ -327,6 +340,24 @@ const char* gdn_last_error(void) { return t_last_error.c_str(); }
 size_t gdn_prefill_workspace_bytes(int n_seqs, int Hv, int dk, int dv, gdn_dtype dtype) {
   if (n_seqs <= 0 || Hv <= 0 || !uses_pc_prefill(dtype, dk, dv)) return 0;
   return gdn::pc::Workspace::bytes(std::min((long)n_seqs * Hv, (long)gdn::pc::kMaxPositions));
+}
+
+gdn_status gdn_prefill_plan(int n_seqs, int64_t total_T, int Hv, int dk, int dv, gdn_dtype dtype, int sm_count_arg,
+                            int* dvp, int* n_chain_ctas, int* rounds) {
+  t_last_error.clear();
+  if (!dvp || !n_chain_ctas || !rounds) return fail(GDN_ERR_INVALID_ARG, "gdn_prefill_plan: null output");
+  if (n_seqs <= 0 || Hv <= 0 || total_T < 0)
+    return fail(GDN_ERR_INVALID_ARG, "gdn_prefill_plan: n_seqs %d, Hv %d, total_T %lld", n_seqs, Hv,
+                (long long)total_T);
+  if (!uses_pc_prefill(dtype, dk, dv))
+    return fail(GDN_ERR_UNSUPPORTED, "gdn_prefill_plan: the tensor-core kernel takes bf16 with dk = dv = 128");
+  const int sms = sm_count_arg > 0 ? sm_count_arg : sm_count();
+  if (sms < 16) return fail(GDN_ERR_INVALID_ARG, "gdn_prefill_plan: %d multiprocessors", sms);
+  const PcLaunchPlan lp = resolve_pc((long)n_seqs * Hv, total_T, n_seqs, Hv, sms);
+  *dvp = lp.dvp;
+  *n_chain_ctas = (int)lp.nc;
+  *rounds = (int)std::min(lp.rounds, (long)INT32_MAX);
+  return GDN_OK;
 }
 
 gdn_status gdn_prefill(const void* q, const void* k, const void* v, const float* g,

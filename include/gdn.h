@@ -84,6 +84,24 @@ int gdn_version(void);
 size_t gdn_prefill_workspace_bytes(int n_seqs, int Hv, int dk, int dv, gdn_dtype dtype);
 
 /*
+ * The launch plan gdn_prefill's tensor-core kernel would use for a problem of
+ * n_seqs sequences, total_T tokens and Hv value heads on a device with
+ * sm_count multiprocessors (0: the current device's): *dvp state rows per
+ * state-carrying CTA (32, 64 or 128), *n_chain_ctas state-carrying CTAs (the
+ * other CTAs prepare packages) and the *rounds in which the sequence-heads
+ * run. The plan comes from the kernel's cost model and the GDN_TC_SLICE /
+ * GDN_PC_NC overrides, with the same clamping a launch applies. Host only:
+ * touches no device memory and launches nothing (with sm_count > 0 it needs
+ * no GPU at all).
+ * Returns GDN_ERR_UNSUPPORTED where the tensor-core kernel does not run
+ * (dtype other than GDN_BF16, or dk, dv other than 128: those shapes run on
+ * the fp32 SIMT kernel) and GDN_ERR_INVALID_ARG for a null output, n_seqs or
+ * Hv <= 0, total_T < 0, or fewer than 16 multiprocessors.
+ */
+gdn_status gdn_prefill_plan(int n_seqs, int64_t total_T, int Hv, int dk, int dv, gdn_dtype dtype, int sm_count,
+                            int* dvp, int* n_chain_ctas, int* rounds);
+
+/*
  * Chunked prefill over packed variable-length sequences.
  *
  *   q, k       [total_T, Hqk, dk]   dtype

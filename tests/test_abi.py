@@ -10,6 +10,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import gated_deltanet_linear_21_b200 as gdn
 from gated_deltanet_linear_21_b200 import build as gdn_build
@@ -115,3 +116,63 @@ def test_workspace_query_is_pure(lib):
     a = lib.gdn_prefill_workspace_bytes(8, 32, 128, 128, gdn.GDN_BF16)
     b = lib.gdn_prefill_workspace_bytes(8, 32, 128, 128, gdn.GDN_BF16)
     assert a == b
+
+
+# ------------------------------------------------------------- launch plan ---
+
+def test_prefill_plan_for_the_benchmark_workloads(monkeypatch):
+    """The cost model's choices (a 148-SM B200 given explicitly: no GPU needed)."""
+    monkeypatch.delenv("GDN_TC_SLICE", raising=False)
+    monkeypatch.delenv("GDN_PC_NC", raising=False)
+    # 4096 tokens x 16 heads: 16 chains of 4 slices of 32 state rows, 84 preparing CTAs
+    assert gdn.prefill_plan(1, 4096, 16, sm_count=148) == (32, 64, 1)
+    # long prompts x 32 heads: 32 chains of one 128-row slice, 116 preparing CTAs
+    assert gdn.prefill_plan(1, 32768, 32, sm_count=148) == (128, 32, 1)
+    assert gdn.prefill_plan(1, 81920, 32, sm_count=148) == (128, 32, 1)
+
+
+@pytest.mark.parametrize("n_seqs,total_T,Hv", [(8, 37000, 32), (300, 45000, 8), (3, 500, 8), (64, 64 * 300, 16)])
+def test_prefill_plan_keeps_rounds_to_whole_sequences(n_seqs, total_T, Hv, monkeypatch):
+    """With several sequences a round runs whole sequences (positions a multiple
+    of Hv) or equal parts of one (a divisor of Hv); every plan leaves CTAs to
+    prepare and covers every sequence-head."""
+    monkeypatch.delenv("GDN_TC_SLICE", raising=False)
+    monkeypatch.delenv("GDN_PC_NC", raising=False)
+    dvp, nc, rounds = gdn.prefill_plan(n_seqs, total_T, Hv, sm_count=148)
+    slices = 128 // dvp
+    positions = nc // slices
+    assert dvp in (32, 64, 128) and nc % slices == 0 and nc <= 148 - 8
+    assert positions % Hv == 0 or Hv % positions == 0
+    assert positions <= min(n_seqs * Hv, 74)
+    assert rounds == -(-(n_seqs * Hv) // positions)
+
+
+def test_prefill_plan_applies_and_clamps_the_overrides(monkeypatch):
+    monkeypatch.setenv("GDN_TC_SLICE", "64")
+    monkeypatch.setenv("GDN_PC_NC", "7")          # rounded down to whole chains of 2 slices
+    assert gdn.prefill_plan(1, 4096, 16, sm_count=148) == (64, 6, 6)
+    monkeypatch.setenv("GDN_PC_NC", "1000")       # no more chain CTAs than slices to run
+    assert gdn.prefill_plan(1, 4096, 16, sm_count=148) == (64, 32, 1)
+    monkeypatch.setenv("GDN_TC_SLICE", "48")      # not a slice width: the model's choice stays
+    monkeypatch.delenv("GDN_PC_NC")
+    assert gdn.prefill_plan(1, 4096, 16, sm_count=148) == (32, 64, 1)
+
+
+def test_prefill_plan_rejects_what_the_kernel_does_not_run(lib, monkeypatch):
+    monkeypatch.delenv("GDN_TC_SLICE", raising=False)
+    monkeypatch.delenv("GDN_PC_NC", raising=False)
+    with pytest.raises(gdn.GdnError) as e:
+        gdn.prefill_plan(1, 4096, 16, dk=64, dv=64, sm_count=148)
+    assert e.value.status == gdn.GDN_ERR_UNSUPPORTED
+    with pytest.raises(gdn.GdnError) as e:
+        gdn.prefill_plan(1, 4096, 16, dtype=torch.float32, sm_count=148)
+    assert e.value.status == gdn.GDN_ERR_UNSUPPORTED
+    for bad in (dict(n_seqs=0), dict(Hv=0), dict(total_T=-1), dict(sm_count=8)):
+        a = dict(n_seqs=1, total_T=4096, Hv=16, sm_count=148)
+        a.update(bad)
+        with pytest.raises(gdn.GdnError) as e:
+            gdn.prefill_plan(a["n_seqs"], a["total_T"], a["Hv"], sm_count=a["sm_count"])
+        assert e.value.status == gdn.GDN_ERR_INVALID_ARG
+    out = ctypes.c_int(0)
+    assert lib.gdn_prefill_plan(1, 4096, 16, 128, 128, gdn.GDN_BF16, 148, None, ctypes.byref(out),
+                                ctypes.byref(out)) == gdn.GDN_ERR_INVALID_ARG
