@@ -164,6 +164,9 @@ def tune_prefill(q, k, v, g, beta, state_in=None, cu_seqlens=None, *, plans=None
     runner = runner or _device_runner
     T, Hqk, dk = q.shape
     Hv, dv = v.shape[1], v.shape[2]
+    if q.dtype != torch.bfloat16 or dk != 128 or dv != 128:
+        raise ValueError("launch plans belong to the tensor-core kernel (bf16, d_k = d_v = 128); "
+                         "other shapes run on the fp32 SIMT kernel, which has none")
     if cu_seqlens is None:
         cu_seqlens = torch.tensor([0, T], dtype=torch.int32, device=q.device)
     N = cu_seqlens.numel() - 1

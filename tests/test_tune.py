@@ -135,3 +135,11 @@ def test_tune_refuses_a_default_plan_that_leaves_elements_unwritten():
 
     with pytest.raises(RuntimeError, match="default plan left state"):
         tune.tune_prefill(q, k, v, g, beta, plans=[(64, 32)], runner=broken)
+
+
+def test_tune_refuses_shapes_without_launch_plans():
+    q, k, v, g, beta = _fake_problem()
+    with pytest.raises(ValueError, match="tensor-core kernel"):
+        tune.tune_prefill(q.float(), k.float(), v.float(), g, beta, plans=[(64, 32)], runner=FakeRunner())
+    with pytest.raises(ValueError, match="tensor-core kernel"):
+        tune.tune_prefill(q[..., :64], k[..., :64], v[..., :64], g, beta, plans=[(64, 32)], runner=FakeRunner())
