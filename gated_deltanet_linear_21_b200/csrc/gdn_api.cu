@@ -333,7 +333,7 @@ gdn_status launch_prefill_pc(const void* q, const void* k, const void* v, const 
 
 extern "C" {
 
-int gdn_version(void) { return (0 << 16) | 2; }
+int gdn_version(void) { return (0 << 16) | 3; }
 
 const char* gdn_last_error(void) { return t_last_error.c_str(); }
 
