@@ -299,3 +299,48 @@ def test_bf16_state_decode_reads_o_before_rounding_and_stores_bf16():
     assert np.array_equal(s16, oracle.round_bf16(s64).reshape(s64.shape))
     assert np.array_equal(s16, oracle.round_bf16(s16).reshape(s16.shape))   # representable
     assert not np.array_equal(s16, s64)
+
+
+# planted mistakes in the bf16 storage path: each must fail a bf16 pin
+
+BF16_MUTANTS = {
+    "bf16_truncates": ("u += 0x7fffu + ((u >> 16) & 1u);", "u += 0u;"),
+    "bf16_ties_away_from_zero": ("u += 0x7fffu + ((u >> 16) & 1u);", "u += 0x8000u;"),
+    "bf16_state_not_rounded": ("if (round_state_bf16) {", "if (0 * round_state_bf16) {"),
+}
+
+
+def _bf16_pins_pass(lib, monkeypatch):
+    dp = ctypes.POINTER(ctypes.c_double)
+    lib.gdn_oracle_decode_ex.restype = ctypes.c_int
+    lib.gdn_oracle_decode_ex.argtypes = [dp] * 6 + [ctypes.c_int] * 5 + [ctypes.c_double] * 2 + \
+        [ctypes.c_int] * 2 + [dp, ctypes.c_int, ctypes.c_int]
+    lib.gdn_oracle_round_bf16.restype = None
+    lib.gdn_oracle_round_bf16.argtypes = [dp, dp, ctypes.c_long]
+    monkeypatch.setattr(oracle, "_lib", lib)
+    try:
+        test_round_bf16_is_round_to_nearest_even_through_float()
+        test_bf16_state_decode_reads_o_before_rounding_and_stores_bf16()
+    except AssertionError:
+        return False
+    return True
+
+
+@pytest.mark.parametrize("name", sorted(BF16_MUTANTS))
+def test_bf16_pins_catch_planted_mistake(name, tmp_path, monkeypatch):
+    src = open(os.path.join(os.path.dirname(oracle.__file__), "gdn_oracle.c")).read()
+    old, new = BF16_MUTANTS[name]
+    assert src.count(old) == 1, f"mutation site for {name} not found"
+    (tmp_path / f"{name}.c").write_text(src.replace(old, new, 1))
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-o", str(tmp_path / f"{name}.so"),
+                    str(tmp_path / f"{name}.c"), "-lm"], check=True)
+    assert not _bf16_pins_pass(ctypes.CDLL(str(tmp_path / f"{name}.so")), monkeypatch), \
+        f"mutant {name} passed the bf16 pins"
+
+
+def test_unmutated_copy_passes_bf16_pins(tmp_path, monkeypatch):
+    src = open(os.path.join(os.path.dirname(oracle.__file__), "gdn_oracle.c")).read()
+    (tmp_path / "same.c").write_text(src)
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-o",
+                    str(tmp_path / "same.so"), str(tmp_path / "same.c"), "-lm"], check=True)
+    assert _bf16_pins_pass(ctypes.CDLL(str(tmp_path / "same.so")), monkeypatch)
