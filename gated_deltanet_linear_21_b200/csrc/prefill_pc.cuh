@@ -64,7 +64,8 @@
 // publishing warp sets ready[q][s mod R] = s / R + 1 with release semantics. A
 // chain's issuing warp waits for that value with acquire semantics and copies
 // the package into shared memory; its releasing warp then adds 1 to
-// consumed[q][s mod R]. Numbers a shorter chain leaves unused are counted as
+// consumed[q][s mod R] (and arrives on the input buffer's free barrier, so that
+// its waits, which go by mbarrier parity, never fall a phase behind). Numbers a shorter chain leaves unused are counted as
 // consumed by its chain CTAs at the end of the round. Items are ordered by (round, chunk, chain), so a prep CTA never waits
 // on a chain that is not running, and the workspace holds P R packages however
 // many sequences there are. Every wait is bounded (~2 s): past it the CTA
