@@ -148,3 +148,109 @@ def test_the_model_reports_the_deadlock_of_uncounted_holes():
     with pytest.raises(AssertionError, match="deadlock"):
         ring_run([3, 20, 20, 20], 2, 2, 4, 3, random.Random(1), bump_holes=False)
     ring_run([3, 20, 20, 20], 2, 2, 4, 3, random.Random(1))
+
+
+# ------------------------------------------------ one chain CTA's mbarriers ---
+
+class MBarrier:
+    """An mbarrier as the kernel uses it: a phase completes when `count` arrivals
+    have been made; a wait on parity P returns once the phase of that parity has
+    completed, which it reads off the parity of the current phase -- so a waiter
+    two phases behind sees its phase as not completed."""
+
+    def __init__(self, count):
+        self.count, self.pending, self.phase = count, count, 0
+
+    def arrive(self):
+        self.pending -= 1
+        if self.pending == 0:
+            self.phase += 1
+            self.pending = self.count
+
+    def test_wait(self, parity):
+        return (self.phase & 1) != parity
+
+
+def chain_cta_run(n_chunks, rng, releasing_warp_arrives=True, max_idle=5000):
+    """The issuing, releasing and compute warps of one chain CTA over two input
+    buffers. A copy lands some time after it is issued (completing bar_full); the
+    releasing warp counts each landed copy once; compute reads each chunk in
+    order. Returns the chunks the releasing warp counted."""
+    full = [MBarrier(1), MBarrier(1)]
+    free = [MBarrier(2 if releasing_warp_arrives else 1) for _ in range(2)]
+    in_flight = []            # buffers whose copy has been issued but has not landed
+    counted = []
+
+    def issuer():
+        for gc in range(n_chunks):
+            b = gc & 1
+            if gc >= 2:
+                while not free[b].test_wait(((gc - 2) >> 1) & 1):
+                    yield "wait"
+            in_flight.append(b)
+            yield "step"
+
+    def lander():             # the asynchronous copies
+        landed = 0
+        while landed < n_chunks:
+            if in_flight and rng.random() < 0.5:
+                full[in_flight.pop(0)].arrive()
+                landed += 1
+                yield "step"
+            else:
+                yield "wait"
+
+    def releaser():
+        for gc in range(n_chunks):
+            b = gc & 1
+            while not full[b].test_wait((gc >> 1) & 1):
+                yield "wait"
+            if releasing_warp_arrives:
+                free[b].arrive()
+            counted.append(gc)
+            yield "step"
+
+    def compute():
+        for gc in range(n_chunks):
+            b = gc & 1
+            while not full[b].test_wait((gc >> 1) & 1):
+                yield "wait"
+            for _ in range(rng.randint(0, 3)):   # the chunk's work
+                yield "step"
+            free[b].arrive()
+            yield "step"
+
+    live = [issuer(), lander(), releaser(), compute()]
+    weights = [1, 1, 1 if releasing_warp_arrives else 0.02, 1]   # a releasing warp that may lag
+    idle = 0
+    while live:
+        k = rng.choices(range(len(live)), weights=weights[:len(live)])[0]
+        try:
+            what = next(live[k])
+        except StopIteration:
+            live.pop(k)
+            weights.pop(k)
+            idle = 0
+            continue
+        idle = idle + 1 if what == "wait" else 0
+        if idle > max_idle:
+            raise AssertionError(f"hang: the releasing warp counted {len(counted)} of {n_chunks} chunks")
+    return counted
+
+
+def test_chain_cta_releasing_warp_never_loses_a_phase():
+    for seed in range(200):
+        assert chain_cta_run(24, random.Random(seed)) == list(range(24))
+
+
+def test_a_releasing_warp_that_does_not_gate_the_buffer_can_lose_a_phase():
+    """Without its arrival on the free barrier, a releasing warp that lags a copy
+    behind waits on a parity that has come round again: it misses that chunk's
+    phase and ends up waiting for a copy that never comes."""
+    hangs = 0
+    for seed in range(60):
+        try:
+            chain_cta_run(24, random.Random(seed), releasing_warp_arrives=False)
+        except AssertionError:
+            hangs += 1
+    assert hangs > 0
