@@ -254,3 +254,102 @@ def test_a_releasing_warp_that_does_not_gate_the_buffer_can_lose_a_phase():
         except AssertionError:
             hangs += 1
     assert hangs > 0
+
+
+# --------------------------------- a prep CTA's queue and its publication ---
+
+def prep_cta_run(n_chunks, P, R, K, rng, publish_when_idle=True, max_idle=20000):
+    """K preparing CTAs and P one-slice chains of n_chunks over a ring of R slots
+    per chain. Each CTA's hand-over warp claims items into a two-entry queue
+    (entry k & 1 is reused once item k - 2 is published) and waits for the
+    item's slot; its compute warps make item `it`'s package and publish it
+    while starting item it + 1 -- or at once if item it + 1 has not been handed
+    over yet (publish_when_idle), since its slot may wait for exactly that
+    package. Returns the chains' reads."""
+    items = [(c, q) for c in range(n_chunks) for q in range(P)]
+    nxt = [0]
+    ready, consumed, slot, reads = {}, {}, {}, []
+    END = object()
+
+    def make_cta():
+        handed, published = {}, set()
+        pending = [None]
+
+        def publish():
+            k = pending[0]
+            c, q = handed[k]
+            key = (q, c % R)
+            slot[key] = c
+            ready[key] = c // R + 1
+            published.add(k)
+            pending[0] = None
+
+        def hand_over():
+            k = 0
+            while True:
+                while k >= 2 and (k - 2) not in published:
+                    yield "wait"
+                if nxt[0] >= len(items):
+                    handed[k] = END
+                    return
+                c, q = items[nxt[0]]
+                nxt[0] += 1
+                while consumed.get((q, c % R), 0) < c // R:
+                    yield "wait"
+                handed[k] = (c, q)
+                k += 1
+                yield "step"
+
+        def compute():
+            it = 0
+            while True:
+                if pending[0] is not None and it not in handed and publish_when_idle:
+                    publish()
+                while it not in handed:
+                    yield "wait"
+                if pending[0] is not None:
+                    publish()
+                if handed[it] is END:
+                    return
+                pending[0] = it
+                it += 1
+                yield "step"
+
+        return [hand_over(), compute()]
+
+    def chain(q):
+        for c in range(n_chunks):
+            key = (q, c % R)
+            while ready.get(key, 0) < c // R + 1:
+                yield "wait"
+            assert slot[key] == c
+            reads.append((q, c))
+            consumed[key] = consumed.get(key, 0) + 1
+            yield "step"
+
+    live = [a for _ in range(K) for a in make_cta()] + [chain(q) for q in range(P)]
+    idle = 0
+    while live:
+        a = rng.choice(live)
+        try:
+            what = next(a)
+        except StopIteration:
+            live.remove(a)
+            idle = 0
+            continue
+        idle = idle + 1 if what == "wait" else 0
+        if idle > max_idle:
+            raise AssertionError("deadlock: a package waits to be published behind its own slot")
+    return reads
+
+
+@pytest.mark.parametrize("P,R,K", [(1, 1, 1), (1, 2, 1), (2, 1, 3), (3, 2, 2), (4, 12, 6)])
+def test_prep_publishes_before_it_can_wait_on_itself(P, R, K):
+    for seed in range(20):
+        reads = prep_cta_run(15, P, R, K, random.Random(seed))
+        assert sorted(reads) == [(q, c) for q in range(P) for c in range(15)]
+
+
+def test_publication_held_until_the_next_item_deadlocks_on_a_small_ring():
+    with pytest.raises(AssertionError, match="deadlock"):
+        prep_cta_run(15, 1, 1, 1, random.Random(0), publish_when_idle=False)
