@@ -143,3 +143,54 @@ def test_tune_refuses_shapes_without_launch_plans():
         tune.tune_prefill(q.float(), k.float(), v.float(), g, beta, plans=[(64, 32)], runner=FakeRunner())
     with pytest.raises(ValueError, match="tensor-core kernel"):
         tune.tune_prefill(q[..., :64], k[..., :64], v[..., :64], g, beta, plans=[(64, 32)], runner=FakeRunner())
+
+
+def test_device_runner_applies_the_plan_times_and_fills_fresh_outputs(monkeypatch):
+    """The device leg's own lines, with the library call, the error check and the
+    CUDA events replaced by stand-ins (no GPU): the plan is in force for every
+    call and undone after, the gated outputs come from a call into NaN-filled
+    buffers, and the time is the events' over the timed calls."""
+    import gated_deltanet_linear_21_b200 as pkg
+    seen = []
+
+    def fake_prefill(q, k, v, g, beta, state_in=None, cu_seqlens=None, *, o=None, state_out=None, **kw):
+        seen.append((os.environ.get("GDN_TC_SLICE"), os.environ.get("GDN_PC_NC"), o is not None))
+        T, Hv, dv = v.shape
+        N = cu_seqlens.numel() - 1
+        if o is not None:
+            assert torch.isnan(o).all() and torch.isnan(state_out).all()   # fresh NaN buffers
+            o.copy_(v.float() * 2)
+            state_out.fill_(3.0)
+            return o, state_out
+        return v * 2, torch.full((N, Hv, dv, q.shape[2]), 3.0)
+
+    class FakeEvent:
+        def __init__(self, enable_timing=False):
+            pass
+
+        def record(self, stream=None):
+            pass
+
+        def elapsed_time(self, other):
+            return 6.0
+
+    monkeypatch.setattr(pkg, "prefill", fake_prefill)
+    monkeypatch.setattr(pkg, "device_error", lambda stream=None: None)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
+    monkeypatch.setattr(torch.cuda, "Event", FakeEvent)
+    monkeypatch.delenv("GDN_TC_SLICE", raising=False)
+    monkeypatch.setenv("GDN_PC_NC", "5")
+    q, k, v, g, beta = _fake_problem()
+    cu = torch.tensor([0, 130], dtype=torch.int32)
+    o, s, ms = tune._device_runner((q, k, v, g, beta, None, cu), (64, 32), 3)
+    assert ms == pytest.approx(2.0)                                   # 6 ms over 3 timed calls
+    assert o.dtype == torch.bfloat16 and o.shape == v.shape and torch.equal(o.float(), (v.float() * 2).to(o.dtype).float())
+    assert s.shape == (1, 4, 128, 128) and bool((s == 3.0).all())
+    assert seen == [("64", "32", False)] * 4 + [("64", "32", True)]  # warm-up, 3 timed, the gated call
+    assert "GDN_TC_SLICE" not in os.environ and os.environ["GDN_PC_NC"] == "5"
+    seen.clear()
+    o, s, ms = tune._device_runner((q, k, v, g, beta, None, cu), None, 0)   # the default plan, untimed
+    assert math.isnan(ms) and seen == [(None, None, True)]
+    # and the whole selection through the device leg
+    best, results = tune.tune_prefill(q, k, v, g, beta, None, cu, plans=[(32, 16), (128, 4)], reps=2)
+    assert all(r.ok for r in results) and (best.dvp, best.nc) == (32, 16)
