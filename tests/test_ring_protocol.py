@@ -353,3 +353,89 @@ def test_prep_publishes_before_it_can_wait_on_itself(P, R, K):
 def test_publication_held_until_the_next_item_deadlocks_on_a_small_ring():
     with pytest.raises(AssertionError, match="deadlock"):
         prep_cta_run(15, 1, 1, 1, random.Random(0), publish_when_idle=False)
+
+
+# ------------------------------ a chain CTA's MMA warp and compute warps ---
+
+def chain_mma_run(n_chunks, rng, max_idle=5000):
+    """The MMA warp and the compute warps of one chain CTA (the compute warps
+    move together: their waits end in a barrier across all eight). Per chunk the
+    MMA warp waits for the input and for the bf16 state copy (bar_s), issues Y and
+    commits it to bar_mma, waits for U_s (bar_u), issues dS and commits it to the
+    same bar_mma; a commit completes when its products finish, some time later.
+    The compute warps wait for Y on bar_mma, stage U_s (bar_u), wait for dS on
+    bar_mma, update the state and write its copy (bar_s). Every wait is by
+    parity. Returns the (chunk, product) pairs the compute warps read."""
+    mma, bar_u, bar_s = MBarrier(1), MBarrier(1), MBarrier(1)
+    issued = []               # products whose commit has not completed yet
+    done = []                 # products completed, in order
+    seen = []
+
+    def mma_warp():
+        ph_s = ph_u = 0
+        for gc in range(n_chunks):
+            while not bar_s.test_wait(ph_s):
+                yield "wait"
+            ph_s ^= 1
+            issued.append((gc, "Y"))
+            yield "step"
+            while not bar_u.test_wait(ph_u):
+                yield "wait"
+            ph_u ^= 1
+            issued.append((gc, "dS"))
+            yield "step"
+
+    def tensor_core():        # commits complete in order, each a while after its issue
+        n = 0
+        while n < 2 * n_chunks:
+            if issued and rng.random() < 0.4:
+                done.append(issued.pop(0))
+                mma.arrive()
+                n += 1
+                yield "step"
+            else:
+                yield "wait"
+
+    def compute():
+        ph = 0
+        bar_s.arrive()        # the first state copy
+        for gc in range(n_chunks):
+            while not mma.test_wait(ph):
+                yield "wait"
+            ph ^= 1
+            seen.append((gc, "Y", done[-1] if done else None))
+            bar_u.arrive()
+            yield "step"
+            while not mma.test_wait(ph):
+                yield "wait"
+            ph ^= 1
+            seen.append((gc, "dS", done[-1] if done else None))
+            if gc + 1 < n_chunks:
+                bar_s.arrive()
+            yield "step"
+
+    live = [mma_warp(), tensor_core(), compute()]
+    idle = 0
+    while live:
+        a = rng.choice(live)
+        try:
+            what = next(a)
+        except StopIteration:
+            live.remove(a)
+            idle = 0
+            continue
+        idle = idle + 1 if what == "wait" else 0
+        if idle > max_idle:
+            raise AssertionError("hang in the chain CTA's MMA handshake")
+    return seen
+
+
+def test_chain_mma_handshake_reads_each_product_once_in_order():
+    """Y and dS share one barrier: the compute warps must see each completion as
+    the product they wait for -- the MMA warp cannot commit the next product
+    before they have seen the last, since it waits on them in between."""
+    for seed in range(200):
+        seen = chain_mma_run(12, random.Random(seed))
+        assert [(g, p) for g, p, _ in seen] == [(g, p) for g in range(12) for p in ("Y", "dS")]
+        for g, p, last_done in seen:
+            assert last_done == (g, p), "a later product completed before this one was read"
