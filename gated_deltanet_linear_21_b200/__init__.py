@@ -7,6 +7,9 @@ no CPU fallback: if the library is missing the import of an op fails loudly.
 
     o, state_out = prefill(q, k, v, g, beta, state_in=None, cu_seqlens=None)
     o = decode(q, k, v, g, beta, state)          # state updated in place
+
+q, k and v may be bf16, f16 or fp32 (all three the same); g, beta and the
+prefill states are fp32.
 """
 from __future__ import annotations
 
@@ -19,15 +22,29 @@ import torch
 __all__ = ["prefill", "prefill_noalloc", "decode", "prefill_workspace_bytes", "prefill_plan", "device_error",
            "wait_selftest",
            "GdnError",
-           "lib", "library_path", "GDN_BF16", "GDN_F32"]
+           "lib", "library_path", "GDN_BF16", "GDN_F32", "GDN_F16"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_PKG, "libgdn.so")
 
 GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_DEVICE_TIMEOUT = range(5)
-GDN_BF16, GDN_F32 = 0, 1
+GDN_BF16, GDN_F32, GDN_F16 = 0, 1, 2
 STATUS_NAMES = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED",
                 3: "GDN_ERR_CUDA", 4: "GDN_ERR_DEVICE_TIMEOUT"}
+
+
+class GdnPlan(ctypes.Structure):
+    """struct gdn_plan: the tensor-core prefill's launch plan (0 = the library's choice)."""
+    _fields_ = [("dvp", ctypes.c_int), ("n_chain_ctas", ctypes.c_int)]
+
+
+def _plan_arg(plan):
+    """A (dvp, n_chain_ctas) pair (None or 0 per field: the library's choice) as a
+    gdn_plan pointer, or None."""
+    if plan is None:
+        return None
+    dvp, nc = plan
+    return ctypes.byref(GdnPlan(int(dvp or 0), int(nc or 0)))
 
 
 class GdnError(RuntimeError):
@@ -54,7 +71,9 @@ SIGNATURES = {
                                  _vp, _fp, _vp]),
     "gdn_device_error": (_i, [_vp]),
     "gdn_wait_selftest": (_i, [_i, _vp]),
-    "gdn_prefill_plan": (_i, [_i, _i64, _i, _i, _i, _i, _i, _vp, _vp, _vp]),
+    "gdn_prefill_ex": (_i, [_vp, _vp, _vp, _fp, _fp, _fp, _i32p, _i, _i64, _i, _i, _i, _i, _f, _i, _i,
+                            _vp, _fp, _vp, _sz, _vp, _vp]),
+    "gdn_prefill_plan": (_i, [_i, _i64, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
 }
 
 
@@ -83,9 +102,46 @@ def _check(status: int):
 def _dtype_code(t: torch.Tensor) -> int:
     if t.dtype == torch.bfloat16:
         return GDN_BF16
+    if t.dtype == torch.float16:
+        return GDN_F16
     if t.dtype == torch.float32:
         return GDN_F32
-    raise TypeError(f"q, k, v must be bf16 or fp32, got {t.dtype}")
+    raise TypeError(f"q, k, v must be bf16, f16 or fp32, got {t.dtype}")
+
+
+def _torch_dtype_code(dtype) -> int:
+    return {torch.bfloat16: GDN_BF16, torch.float16: GDN_F16, torch.float32: GDN_F32}[dtype]
+
+
+def _shape(t, name, shape):
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _prefill_args(q, k, v, g, beta, state_in, cu_seqlens, o, state_out):
+    """Checks and default outputs shared by the prefill entry points."""
+    _dev(q, "q"); _dev(k, "k", q.dtype); _dev(v, "v", q.dtype)
+    _dev(g, "g", torch.float32); _dev(beta, "beta", torch.float32)
+    if q.dim() != 3 or v.dim() != 3:
+        raise ValueError("q, k must be [T, Hqk, dk] and v [T, Hv, dv]")
+    T, Hqk, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[2]
+    _shape(k, "k", (T, Hqk, dk)); _shape(v, "v", (T, Hv, dv))
+    _shape(g, "g", (T, Hv)); _shape(beta, "beta", (T, Hv))
+    if cu_seqlens is None:
+        cu_seqlens = torch.tensor([0, T], dtype=torch.int32, device=q.device)
+    _dev(cu_seqlens, "cu_seqlens", torch.int32)
+    N = cu_seqlens.numel() - 1
+    if state_in is not None:
+        _dev(state_in, "state_in", torch.float32)
+        _shape(state_in, "state_in", (N, Hv, dv, dk))
+    if o is None:
+        o = torch.empty(T, Hv, dv, dtype=q.dtype, device=q.device)
+    _dev(o, "o", q.dtype); _shape(o, "o", (T, Hv, dv))
+    if state_out is None:
+        state_out = torch.empty(N, Hv, dv, dk, dtype=torch.float32, device=q.device)
+    _dev(state_out, "state_out", torch.float32); _shape(state_out, "state_out", (N, Hv, dv, dk))
+    return T, Hqk, dk, Hv, dv, N, cu_seqlens, o, state_out
 
 
 def _dev(t, name, dtype=None):
@@ -104,53 +160,41 @@ def _stream_handle(stream) -> int:
 
 
 def prefill_workspace_bytes(n_seqs, Hv, dk, dv, dtype=torch.bfloat16) -> int:
-    code = GDN_BF16 if dtype == torch.bfloat16 else GDN_F32
-    return int(lib().gdn_prefill_workspace_bytes(n_seqs, Hv, dk, dv, code))
+    return int(lib().gdn_prefill_workspace_bytes(n_seqs, Hv, dk, dv, _torch_dtype_code(dtype)))
 
 
-def prefill_plan(n_seqs, total_T, Hv, dk=128, dv=128, dtype=torch.bfloat16, sm_count=0):
+def prefill_plan(n_seqs, total_T, Hv, dk=128, dv=128, dtype=torch.bfloat16, sm_count=0, requested=None):
     """(dvp, n_chain_ctas, rounds): the launch plan the tensor-core prefill would
-    use for this problem (the GDN_TC_SLICE / GDN_PC_NC overrides included);
+    use for this problem, given a `requested` (dvp, n_chain_ctas) plan or None;
     host only. sm_count=0 asks the current device."""
-    code = GDN_BF16 if dtype == torch.bfloat16 else GDN_F32
     out = [ctypes.c_int(0) for _ in range(3)]
-    _check(lib().gdn_prefill_plan(int(n_seqs), int(total_T), int(Hv), int(dk), int(dv), code, int(sm_count),
-                                  *[ctypes.byref(x) for x in out]))
+    _check(lib().gdn_prefill_plan(int(n_seqs), int(total_T), int(Hv), int(dk), int(dv), _torch_dtype_code(dtype),
+                                  int(sm_count), _plan_arg(requested), *[ctypes.byref(x) for x in out]))
     return tuple(x.value for x in out)
 
 
 def prefill(q, k, v, g, beta, state_in=None, cu_seqlens=None, *, scale=None, chunk=0,
-            o=None, state_out=None, workspace=None, stream=None):
+            o=None, state_out=None, workspace=None, plan=None, stream=None):
     """Chunked prefill over packed sequences.
 
-    q, k [T, Hqk, dk]; v [T, Hv, dv] (bf16 or fp32, same dtype); g, beta [T, Hv]
-    fp32; state_in [N, Hv, dv, dk] fp32 or None; cu_seqlens [N+1] int32 (None =
-    one sequence of T tokens). Returns (o [T, Hv, dv], state_out [N, Hv, dv, dk]).
+    q, k [T, Hqk, dk]; v [T, Hv, dv] (bf16, f16 or fp32, same dtype); g, beta
+    [T, Hv] fp32; state_in [N, Hv, dv, dk] fp32 or None; cu_seqlens [N+1] int32
+    (None = one sequence of T tokens). `plan` = (dvp, n_chain_ctas) for the
+    tensor-core kernel (gdn_prefill_ex; None or 0: the library's choice).
+    Returns (o [T, Hv, dv], state_out [N, Hv, dv, dk]).
     """
-    _dev(q, "q"); _dev(k, "k", q.dtype); _dev(v, "v", q.dtype)
-    _dev(g, "g", torch.float32); _dev(beta, "beta", torch.float32)
-    T, Hqk, dk = q.shape
-    Hv, dv = v.shape[1], v.shape[2]
-    if cu_seqlens is None:
-        cu_seqlens = torch.tensor([0, T], dtype=torch.int32, device=q.device)
-    _dev(cu_seqlens, "cu_seqlens", torch.int32)
-    N = cu_seqlens.numel() - 1
-    if state_in is not None:
-        _dev(state_in, "state_in", torch.float32)
-    if o is None:
-        o = torch.empty(T, Hv, dv, dtype=q.dtype, device=q.device)
-    if state_out is None:
-        state_out = torch.empty(N, Hv, dv, dk, dtype=torch.float32, device=q.device)
+    T, Hqk, dk, Hv, dv, N, cu_seqlens, o, state_out = _prefill_args(q, k, v, g, beta, state_in, cu_seqlens,
+                                                                    o, state_out)
     need = prefill_workspace_bytes(N, Hv, dk, dv, q.dtype)
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_ptr = workspace.data_ptr() if workspace is not None else None
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    _check(lib().gdn_prefill(
+    _check(lib().gdn_prefill_ex(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), g.data_ptr(), beta.data_ptr(),
         state_in.data_ptr() if state_in is not None else None, cu_seqlens.data_ptr(),
         N, T, Hqk, Hv, dk, dv, float(scale or 0.0), int(chunk), _dtype_code(q),
-        o.data_ptr(), state_out.data_ptr(), ws_ptr, ws_bytes, _stream_handle(stream)))
+        o.data_ptr(), state_out.data_ptr(), ws_ptr, ws_bytes, _plan_arg(plan), _stream_handle(stream)))
     return o, state_out
 
 
@@ -159,18 +203,8 @@ def prefill_noalloc(q, k, v, g, beta, state_in=None, cu_seqlens=None, *, scale=N
     """gdn_prefill_noalloc: the prefill with the library's built-in scratch
     instead of a workspace (for callers that cannot allocate device memory).
     Outputs are allocated here only if not given."""
-    _dev(q, "q"); _dev(k, "k", q.dtype); _dev(v, "v", q.dtype)
-    _dev(g, "g", torch.float32); _dev(beta, "beta", torch.float32)
-    T, Hqk, dk = q.shape
-    Hv, dv = v.shape[1], v.shape[2]
-    if cu_seqlens is None:
-        cu_seqlens = torch.tensor([0, T], dtype=torch.int32, device=q.device)
-    _dev(cu_seqlens, "cu_seqlens", torch.int32)
-    N = cu_seqlens.numel() - 1
-    if o is None:
-        o = torch.empty(T, Hv, dv, dtype=q.dtype, device=q.device)
-    if state_out is None:
-        state_out = torch.empty(N, Hv, dv, dk, dtype=torch.float32, device=q.device)
+    T, Hqk, dk, Hv, dv, N, cu_seqlens, o, state_out = _prefill_args(q, k, v, g, beta, state_in, cu_seqlens,
+                                                                    o, state_out)
     _check(lib().gdn_prefill_noalloc(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), g.data_ptr(), beta.data_ptr(),
         state_in.data_ptr() if state_in is not None else None, cu_seqlens.data_ptr(),

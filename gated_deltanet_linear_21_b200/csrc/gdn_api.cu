@@ -17,7 +17,6 @@
 #include "prefill_pc.cuh"
 
 #include <cudaTypedefs.h>
-#include <cstdlib>
 
 namespace {
 
@@ -150,15 +149,17 @@ gdn_status launch_prefill_simt(const void* q, const void* k, const void* v, cons
 }
 
 // ------------------------------------------------- tensor-core prefill ---
+// The driver's tensor-map encoder, looked up once per process (thread-safe).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static std::once_flag once;
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
+  std::call_once(once, [] {
     cudaDriverEntryPointQueryResult q;
     void* p = nullptr;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
       fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
+  });
   return fn;
 }
 
@@ -269,22 +270,29 @@ PcPlan plan_pc(long chains, int64_t total_T, int n_seqs, int Hv, int sms) {
   return best;
 }
 
-// The plan a launch uses: the model's choice, then the GDN_TC_SLICE / GDN_PC_NC
-// overrides, clamped so that no position is without a chain, a chain's slices
-// stay in one round and the package ring's positions suffice.
+// The plan a launch uses: the model's choice, replaced field by field by the
+// caller's request (a field of 0 keeps the model's value), clamped so that no
+// position is without a chain, a chain's slices stay in one round and the
+// package ring's positions suffice. The request is validated by the caller.
 struct PcLaunchPlan {
   int dvp;
   long nc, rounds;
 };
-PcLaunchPlan resolve_pc(long chains, int64_t total_T, int n_seqs, int Hv, int sms) {
+bool plan_request_ok(const gdn_plan* req) {
+  if (!req) return true;
+  return (req->dvp == 0 || req->dvp == 32 || req->dvp == 64 || req->dvp == 128) && req->n_chain_ctas >= 0;
+}
+PcLaunchPlan resolve_pc(long chains, int64_t total_T, int n_seqs, int Hv, int sms, const gdn_plan* req) {
   PcPlan plan = plan_pc(chains, total_T, n_seqs, Hv, sms);
-  if (const char* env = getenv("GDN_TC_SLICE")) {
-    const int v2 = atoi(env);
-    if (v2 == 32 || v2 == 64 || v2 == 128) plan.dvp = v2;
+  if (req && req->dvp != 0 && req->dvp != plan.dvp) {
+    // another slice width: keep the model's number of chains per round
+    plan.nc = plan.nc / (128 / plan.dvp) * (128 / req->dvp);
+    plan.dvp = req->dvp;
   }
   const int dvp = plan.dvp, slices = 128 / dvp;
   long nc = plan.nc;
-  if (const char* env = getenv("GDN_PC_NC")) nc = std::max(1, std::min(atoi(env), sms - 1));
+  if (req && req->n_chain_ctas > 0) nc = std::max(1, std::min(req->n_chain_ctas, sms - 1));
+  nc = std::min(nc, (long)sms - 1);
   nc = std::min(nc, chains * slices);
   nc = std::min(nc, (long)gdn::pc::kMaxPositions * slices);
   nc -= nc % slices;
@@ -294,11 +302,12 @@ PcLaunchPlan resolve_pc(long chains, int64_t total_T, int n_seqs, int Hv, int sm
 
 gdn_status launch_prefill_pc(const void* q, const void* k, const void* v, const float* g, const float* beta,
                              const float* state_in, const int32_t* cu, int n_seqs, int64_t total_T, int Hqk,
-                             int Hv, float scale, void* o, float* state_out, void* ws, cudaStream_t st) {
+                             int Hv, float scale, void* o, float* state_out, void* ws, const gdn_plan* req,
+                             cudaStream_t st) {
   const long chains = (long)n_seqs * Hv;
   const int sms = sm_count();
   if (sms < 16) return fail(GDN_ERR_CUDA, "gdn_prefill: cannot query the multiprocessor count");
-  const PcLaunchPlan lp = resolve_pc(chains, total_T, n_seqs, Hv, sms);
+  const PcLaunchPlan lp = resolve_pc(chains, total_T, n_seqs, Hv, sms, req);
   const int dvp = lp.dvp, slices = 128 / dvp;
   const long nc = lp.nc;
   if (lp.rounds > gdn::pc::kMaxRounds)
@@ -343,9 +352,12 @@ size_t gdn_prefill_workspace_bytes(int n_seqs, int Hv, int dk, int dv, gdn_dtype
 }
 
 gdn_status gdn_prefill_plan(int n_seqs, int64_t total_T, int Hv, int dk, int dv, gdn_dtype dtype, int sm_count_arg,
-                            int* dvp, int* n_chain_ctas, int* rounds) {
+                            const gdn_plan* requested, int* dvp, int* n_chain_ctas, int* rounds) {
   t_last_error.clear();
   if (!dvp || !n_chain_ctas || !rounds) return fail(GDN_ERR_INVALID_ARG, "gdn_prefill_plan: null output");
+  if (!plan_request_ok(requested))
+    return fail(GDN_ERR_INVALID_ARG, "gdn_prefill_plan: requested dvp %d (0, 32, 64 or 128), n_chain_ctas %d (>= 0)",
+                requested->dvp, requested->n_chain_ctas);
   if (n_seqs <= 0 || Hv <= 0 || total_T < 0)
     return fail(GDN_ERR_INVALID_ARG, "gdn_prefill_plan: n_seqs %d, Hv %d, total_T %lld", n_seqs, Hv,
                 (long long)total_T);
@@ -353,18 +365,21 @@ gdn_status gdn_prefill_plan(int n_seqs, int64_t total_T, int Hv, int dk, int dv,
     return fail(GDN_ERR_UNSUPPORTED, "gdn_prefill_plan: the tensor-core kernel takes bf16 with dk = dv = 128");
   const int sms = sm_count_arg > 0 ? sm_count_arg : sm_count();
   if (sms < 16) return fail(GDN_ERR_INVALID_ARG, "gdn_prefill_plan: %d multiprocessors", sms);
-  const PcLaunchPlan lp = resolve_pc((long)n_seqs * Hv, total_T, n_seqs, Hv, sms);
+  const PcLaunchPlan lp = resolve_pc((long)n_seqs * Hv, total_T, n_seqs, Hv, sms, requested);
   *dvp = lp.dvp;
   *n_chain_ctas = (int)lp.nc;
   *rounds = (int)std::min(lp.rounds, (long)INT32_MAX);
   return GDN_OK;
 }
 
-gdn_status gdn_prefill(const void* q, const void* k, const void* v, const float* g,
-                       const float* beta, const float* state_in, const int32_t* cu_seqlens,
-                       int n_seqs, int64_t total_T, int Hqk, int Hv, int dk, int dv, float scale,
-                       int chunk, gdn_dtype dtype, void* o, float* state_out, void* workspace,
-                       size_t workspace_bytes, void* stream) {
+gdn_status gdn_prefill_ex(const void* q, const void* k, const void* v, const float* g,
+                          const float* beta, const float* state_in, const int32_t* cu_seqlens,
+                          int n_seqs, int64_t total_T, int Hqk, int Hv, int dk, int dv, float scale,
+                          int chunk, gdn_dtype dtype, void* o, float* state_out, void* workspace,
+                          size_t workspace_bytes, const gdn_plan* plan, void* stream) {
+  if (!plan_request_ok(plan))
+    return fail(GDN_ERR_INVALID_ARG, "gdn_prefill: plan dvp %d (0, 32, 64 or 128), n_chain_ctas %d (>= 0)",
+                plan->dvp, plan->n_chain_ctas);
   if (n_seqs < 0) return fail(GDN_ERR_INVALID_ARG, "gdn_prefill: n_seqs=%d < 0", n_seqs);
   if (total_T < 0 || total_T >= (int64_t(1) << 31))
     return fail(GDN_ERR_INVALID_ARG, "gdn_prefill: total_T=%lld out of range", (long long)total_T);
@@ -396,12 +411,21 @@ gdn_status gdn_prefill(const void* q, const void* k, const void* v, const float*
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (uses_pc_prefill(dtype, dk, dv) && C == 64 && total_T > 0)
     return launch_prefill_pc(q, k, v, g, beta, state_in, cu_seqlens, n_seqs, total_T, Hqk, Hv, scale, o, state_out,
-                             workspace, st);
+                             workspace, plan, st);
   if (dtype == GDN_F32)
     return launch_prefill_simt<float>(q, k, v, g, beta, state_in, cu_seqlens, n_seqs, total_T, Hqk,
                                       Hv, dk, dv, scale, C, o, state_out, st);
   return launch_prefill_simt<__nv_bfloat16>(q, k, v, g, beta, state_in, cu_seqlens, n_seqs, total_T,
                                             Hqk, Hv, dk, dv, scale, C, o, state_out, st);
+}
+
+gdn_status gdn_prefill(const void* q, const void* k, const void* v, const float* g,
+                       const float* beta, const float* state_in, const int32_t* cu_seqlens,
+                       int n_seqs, int64_t total_T, int Hqk, int Hv, int dk, int dv, float scale,
+                       int chunk, gdn_dtype dtype, void* o, float* state_out, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  return gdn_prefill_ex(q, k, v, g, beta, state_in, cu_seqlens, n_seqs, total_T, Hqk, Hv, dk, dv, scale, chunk,
+                        dtype, o, state_out, workspace, workspace_bytes, nullptr, stream);
 }
 
 gdn_status gdn_decode(const void* q, const void* k, const void* v, const float* g,
@@ -474,11 +498,15 @@ gdn_status gdn_device_error(void* stream) {
 // memory and gdn_prefill_noalloc runs the same kernel on it.
 //
 // The array lives as long as the library is loaded, on every device that
-// loads it. Its device address is looked up once per device (first call with
-// that device current) with cudaGetSymbolAddress; host code must never use
-// the array's name as a device pointer. Every call shares the array: the
-// parts that must start at zero are cleared by each call on its stream, and
-// two calls whose kernels overlap on the GPU (different streams, or different
+// loads it. Host code must never use the array's name as a device pointer:
+// its device address is looked up with cudaGetSymbolAddress, with the device
+// current. The address belongs to the CUDA context the module was loaded in,
+// so it is cached per device together with that context's id and looked up
+// again on every call made outside stream capture (a cheap host-side query);
+// a call under capture uses the cached address, which must come from an
+// earlier call in the same context. Every call shares the array: the parts
+// that must start at zero are cleared by each call on its stream, and two
+// calls whose kernels overlap on the GPU (different streams, or different
 // host threads) race on it and must be serialised by the caller.
 // ============================================================================
 namespace {
@@ -490,25 +518,63 @@ constexpr size_t kNoAllocScratchBytes =
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
+struct NoAllocAddr {
+  unsigned long long ctx_id;   // the context the address was looked up in
+  void* ptr;
+};
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {};
+NoAllocAddr g_noalloc_addr[kMaxDevices] = {};
 
-gdn_status noalloc_scratch(void** out) {
+// Id of the calling thread's current CUDA context (driver entry points looked
+// up once); false if there is none or the driver lacks the query.
+bool current_context_id(unsigned long long* id) {
+  static std::once_flag once;
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  if (!get_current || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+gdn_status noalloc_scratch(cudaStream_t st, void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "gdn_prefill_noalloc: %s", cudaGetErrorString(e));
   if (dev < 0 || dev >= kMaxDevices)
     return fail(GDN_ERR_UNSUPPORTED, "gdn_prefill_noalloc: device %d beyond %d", dev, kMaxDevices);
+  // (a runtime call on the stream also makes the device's context current)
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(st, &cap);
+  if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "gdn_prefill_noalloc: %s", cudaGetErrorString(e));
+  unsigned long long ctx = 0;
+  if (!current_context_id(&ctx))
+    return fail(GDN_ERR_CUDA, "gdn_prefill_noalloc: cannot identify the current CUDA context");
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  NoAllocAddr& a = g_noalloc_addr[dev];
+  if (cap == cudaStreamCaptureStatusNone) {
     void* ptr = nullptr;
     e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
     if (e != cudaSuccess || !ptr)
-      return fail(GDN_ERR_CUDA, "gdn_prefill_noalloc: cudaGetSymbolAddress failed: %s",
-                  cudaGetErrorString(e));
-    g_noalloc_ptr[dev] = ptr;
+      return fail(GDN_ERR_CUDA, "gdn_prefill_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
+    a = {ctx, ptr};
+  } else if (!a.ptr || a.ctx_id != ctx) {
+    return fail(GDN_ERR_CUDA,
+                "gdn_prefill_noalloc: called under stream capture before any call outside capture in this "
+                "CUDA context (the scratch address is looked up outside capture)");
   }
-  *out = g_noalloc_ptr[dev];
+  *out = a.ptr;
   return GDN_OK;
 }
 
@@ -531,7 +597,7 @@ extern "C" gdn_status gdn_prefill_noalloc(const void* q, const void* k, const vo
                   n_seqs, Hv, need, kNoAllocScratchBytes);
   }
   void* scratch = nullptr;
-  if (gdn_status s = noalloc_scratch(&scratch)) return s;
+  if (gdn_status s = noalloc_scratch(static_cast<cudaStream_t>(stream), &scratch)) return s;
   return gdn_prefill(q, k, v, g, beta, state_in, cu_seqlens, n_seqs, total_T, Hqk, Hv, dk, dv, scale, chunk,
                      dtype, o, state_out, scratch, kNoAllocScratchBytes, stream);
 }

@@ -9,29 +9,27 @@ compiler on Apple's chips", section "The night the engine chose wrong": each
 candidate is compared with a kernel already trusted, on a full and a partial
 block, and dropped beyond 1/64 of the largest value):
 
-* each candidate plan runs the caller's problem through the library's plan
-  overrides (the GDN_TC_SLICE / GDN_PC_NC environment variables read at every
-  call), timed with CUDA events over a few calls after a warm-up;
+* each candidate plan runs the caller's problem with that plan passed to the
+  call (gdn_prefill_ex), timed with CUDA events over a few calls after a
+  warm-up;
 * its outputs must match the default plan's within 1/64 of the largest value,
   on the caller's problem and on a check problem of one full and one partial
   64-token chunk entering a non-zero state. The pages zero the output first;
   here it is filled with NaN, which shows an unwritten element whatever value
   was expected there;
-* the fastest plan that passes is returned; ``plan_override`` applies it.
+* the fastest plan that passes is returned; pass ``(best.dvp, best.nc)`` as
+  ``plan=`` to ``prefill`` to run with it.
 
 Only the plan differs between candidates: every run goes through the library's
 kernels, and the default plan is the one the parity tests hold to the oracle.
 """
 from __future__ import annotations
 
-import contextlib
 import math
-import os
 from dataclasses import dataclass
 
 import torch
 
-_ENV = ("GDN_TC_SLICE", "GDN_PC_NC")
 _SLICE_WIDTHS = (32, 64, 128)
 
 
@@ -43,26 +41,6 @@ class PlanResult:
     err: float         # largest difference from the default plan (o, state, check problem)
     ok: bool
     reason: str = ""
-
-
-@contextlib.contextmanager
-def plan_override(dvp=None, nc=None):
-    """Run the enclosed prefill calls with slice width `dvp` and `nc` state-carrying
-    CTAs (None: the library's own choice); the environment is restored after."""
-    old = {k: os.environ.get(k) for k in _ENV}
-    try:
-        for key, val in zip(_ENV, (dvp, nc)):
-            if val:
-                os.environ[key] = str(int(val))
-            else:
-                os.environ.pop(key, None)
-        yield
-    finally:
-        for key, val in old.items():
-            if val is None:
-                os.environ.pop(key, None)
-            else:
-                os.environ[key] = val
 
 
 def candidate_plans(n_chains: int, sms: int = 148, max_positions: int = 74):
@@ -135,23 +113,21 @@ def _device_runner(args, plan, reps):
     T, _, dk = q.shape
     Hv, dv = v.shape[1], v.shape[2]
     N = cu.numel() - 1
-    dvp, nc = plan if plan else (None, None)
-    with plan_override(dvp, nc):
-        ms = math.nan
-        if reps > 0:
-            prefill(q, k, v, g, beta, state_in, cu)   # warm-up
-            torch.cuda.synchronize()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()
-            for _ in range(reps):
-                prefill(q, k, v, g, beta, state_in, cu)
-            b.record()
-            torch.cuda.synchronize()
-            ms = a.elapsed_time(b) / reps
-        o = torch.full((T, Hv, dv), math.nan, dtype=q.dtype, device=q.device)
-        s = torch.full((N, Hv, dv, dk), math.nan, dtype=torch.float32, device=q.device)
-        prefill(q, k, v, g, beta, state_in, cu, o=o, state_out=s)
-        device_error()
+    ms = math.nan
+    if reps > 0:
+        prefill(q, k, v, g, beta, state_in, cu, plan=plan)   # warm-up
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            prefill(q, k, v, g, beta, state_in, cu, plan=plan)
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / reps
+    o = torch.full((T, Hv, dv), math.nan, dtype=q.dtype, device=q.device)
+    s = torch.full((N, Hv, dv, dk), math.nan, dtype=torch.float32, device=q.device)
+    prefill(q, k, v, g, beta, state_in, cu, o=o, state_out=s, plan=plan)
+    device_error()
     return o, s, ms
 
 

@@ -67,6 +67,21 @@ typedef enum gdn_dtype {
     GDN_F32 = 1
 } gdn_dtype;
 
+/*
+ * Launch plan of the tensor-core prefill (bf16, dk = dv = 128). The kernel
+ * splits its CTAs into ones that carry the recurrence state from chunk to
+ * chunk, each owning a slice of `dvp` state rows of one (sequence, value head)
+ * at a time, and ones that prepare the chunks' state-independent operands.
+ * A field of 0 keeps the library's choice (a cost model of the two sides);
+ * dvp must be 0, 32, 64 or 128 and n_chain_ctas >= 0. A requested plan is
+ * clamped as gdn_prefill_plan documents. The result does not depend on the
+ * plan beyond rounding.
+ */
+typedef struct gdn_plan {
+    int dvp;            /* state rows per state-carrying CTA: 32, 64, 128 (0: the model's) */
+    int n_chain_ctas;   /* number of state-carrying CTAs (0: the model's) */
+} gdn_plan;
+
 /* Library version, (major << 16) | minor. */
 int gdn_version(void);
 
@@ -84,22 +99,24 @@ int gdn_version(void);
 size_t gdn_prefill_workspace_bytes(int n_seqs, int Hv, int dk, int dv, gdn_dtype dtype);
 
 /*
- * The launch plan gdn_prefill's tensor-core kernel would use for a problem of
- * n_seqs sequences, total_T tokens and Hv value heads on a device with
- * sm_count multiprocessors (0: the current device's): *dvp state rows per
- * state-carrying CTA (32, 64 or 128), *n_chain_ctas state-carrying CTAs (the
- * other CTAs prepare packages) and the *rounds in which the sequence-heads
- * run. The plan comes from the kernel's cost model and the GDN_TC_SLICE /
- * GDN_PC_NC overrides, with the same clamping a launch applies. Host only:
- * touches no device memory and launches nothing (with sm_count > 0 it needs
- * no GPU at all).
+ * The launch plan gdn_prefill_ex's tensor-core kernel would use for a problem
+ * of n_seqs sequences, total_T tokens and Hv value heads on a device with
+ * sm_count multiprocessors (0: the current device's), given the `requested`
+ * plan (NULL: none): *dvp state rows per state-carrying CTA (32, 64 or 128),
+ * *n_chain_ctas state-carrying CTAs (the other CTAs prepare packages) and the
+ * *rounds in which the sequence-heads run. Clamping, as a launch applies it:
+ * a requested dvp without a CTA count keeps the model's chains per round; the
+ * count is capped at sm_count - 1, at the slices there are to run and at 74
+ * chains at a time, and rounded down to whole chains (at least one).
+ * Host only: touches no device memory and launches nothing (with sm_count > 0
+ * it needs no GPU at all).
  * Returns GDN_ERR_UNSUPPORTED where the tensor-core kernel does not run
  * (dtype other than GDN_BF16, or dk, dv other than 128: those shapes run on
- * the fp32 SIMT kernel) and GDN_ERR_INVALID_ARG for a null output, n_seqs or
- * Hv <= 0, total_T < 0, or fewer than 16 multiprocessors.
+ * the fp32 SIMT kernel) and GDN_ERR_INVALID_ARG for a null output, an invalid
+ * request, n_seqs or Hv <= 0, total_T < 0, or fewer than 16 multiprocessors.
  */
 gdn_status gdn_prefill_plan(int n_seqs, int64_t total_T, int Hv, int dk, int dv, gdn_dtype dtype, int sm_count,
-                            int* dvp, int* n_chain_ctas, int* rounds);
+                            const gdn_plan *requested, int *dvp, int *n_chain_ctas, int *rounds);
 
 /*
  * Chunked prefill over packed variable-length sequences.
@@ -126,10 +143,8 @@ gdn_status gdn_prefill_plan(int n_seqs, int64_t total_T, int Hv, int dk, int dv,
  * across calls). It is one cooperative launch with one CTA on every SM of the
  * device: other work on the device runs before or after it, not beside it.
  * How it splits the work (the width of the state slices and the number of
- * CTAs that carry states) is chosen from the problem's shape; for experiments
- * the environment variables GDN_TC_SLICE (32, 64 or 128 state rows) and
- * GDN_PC_NC (number of state-carrying CTAs) override the choice. The result
- * does not depend on either beyond rounding.
+ * CTAs that carry states) is chosen from the problem's shape; gdn_prefill_ex
+ * takes an explicit plan instead.
  * cu_seqlens is read on the device only; a cu_seqlens that breaks the rules
  * above is not detected on the host -- sequences with negative length are
  * treated as empty and tokens outside [0, total_T) are never read.
@@ -141,6 +156,23 @@ gdn_status gdn_prefill(const void *q, const void *k, const void *v,
                        float scale, int chunk, gdn_dtype dtype,
                        void *o, float *state_out,
                        void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * gdn_prefill with an explicit launch plan for the tensor-core kernel (see
+ * gdn_plan; NULL or zero fields: the library's choice, so that
+ * gdn_prefill(...) is gdn_prefill_ex(..., NULL, stream)). The plan is an
+ * argument of the call, not process state: concurrent calls from several host
+ * threads each run their own. Ignored by the fp32 SIMT kernel. An invalid plan
+ * returns GDN_ERR_INVALID_ARG before anything is enqueued.
+ */
+gdn_status gdn_prefill_ex(const void *q, const void *k, const void *v,
+                          const float *g, const float *beta,
+                          const float *state_in, const int32_t *cu_seqlens,
+                          int n_seqs, int64_t total_T, int Hqk, int Hv, int dk, int dv,
+                          float scale, int chunk, gdn_dtype dtype,
+                          void *o, float *state_out,
+                          void *workspace, size_t workspace_bytes,
+                          const gdn_plan *plan, void *stream);
 
 /*
  * Allocation-free variant of gdn_prefill for callers that cannot provide
@@ -159,9 +191,14 @@ gdn_status gdn_prefill(const void *q, const void *k, const void *v,
  *   Supported: GDN_BF16, dk = dv = 128, chunk 0 or 64 (anything else returns
  *   GDN_ERR_UNSUPPORTED); every problem size gdn_prefill accepts fits the
  *   array.
- *   The first call on each device looks up the array's device address with
- *   cudaGetSymbolAddress (with that device current); make that first call
- *   before capturing the stream into a CUDA graph.
+ *   The array's device address belongs to the CUDA context the library's
+ *   module is loaded in. Every call made outside stream capture looks it up
+ *   with cudaGetSymbolAddress (with the calling thread's device current) and
+ *   caches it with that context's id; a call under stream capture uses the
+ *   cached address, so make a first call outside capture in that context
+ *   before capturing a stream into a CUDA graph (otherwise GDN_ERR_CUDA).
+ *   A context that was destroyed and created again (cudaDeviceReset) is
+ *   recognised by its new id.
  *   All calls share the one array and each call clears the part that must
  *   start at zero on its stream: calls whose kernels can overlap on the GPU
  *   (different streams or host threads) race and must be serialised by the

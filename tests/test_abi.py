@@ -120,10 +120,8 @@ def test_workspace_query_is_pure(lib):
 
 # ------------------------------------------------------------- launch plan ---
 
-def test_prefill_plan_for_the_benchmark_workloads(monkeypatch):
+def test_prefill_plan_for_the_benchmark_workloads():
     """The cost model's choices (a 148-SM B200 given explicitly: no GPU needed)."""
-    monkeypatch.delenv("GDN_TC_SLICE", raising=False)
-    monkeypatch.delenv("GDN_PC_NC", raising=False)
     # 4096 tokens x 16 heads: 16 chains of 4 slices of 32 state rows, 84 preparing CTAs
     assert gdn.prefill_plan(1, 4096, 16, sm_count=148) == (32, 64, 1)
     # long prompts x 32 heads: 32 chains of one 128-row slice, 116 preparing CTAs
@@ -132,12 +130,10 @@ def test_prefill_plan_for_the_benchmark_workloads(monkeypatch):
 
 
 @pytest.mark.parametrize("n_seqs,total_T,Hv", [(8, 37000, 32), (300, 45000, 8), (3, 500, 8), (64, 64 * 300, 16)])
-def test_prefill_plan_keeps_rounds_to_whole_sequences(n_seqs, total_T, Hv, monkeypatch):
+def test_prefill_plan_keeps_rounds_to_whole_sequences(n_seqs, total_T, Hv):
     """With several sequences a round runs whole sequences (positions a multiple
     of Hv) or equal parts of one (a divisor of Hv); every plan leaves CTAs to
     prepare and covers every sequence-head."""
-    monkeypatch.delenv("GDN_TC_SLICE", raising=False)
-    monkeypatch.delenv("GDN_PC_NC", raising=False)
     dvp, nc, rounds = gdn.prefill_plan(n_seqs, total_T, Hv, sm_count=148)
     slices = 128 // dvp
     positions = nc // slices
@@ -147,20 +143,51 @@ def test_prefill_plan_keeps_rounds_to_whole_sequences(n_seqs, total_T, Hv, monke
     assert rounds == -(-(n_seqs * Hv) // positions)
 
 
-def test_prefill_plan_applies_and_clamps_the_overrides(monkeypatch):
-    monkeypatch.setenv("GDN_TC_SLICE", "64")
-    monkeypatch.setenv("GDN_PC_NC", "7")          # rounded down to whole chains of 2 slices
-    assert gdn.prefill_plan(1, 4096, 16, sm_count=148) == (64, 6, 6)
-    monkeypatch.setenv("GDN_PC_NC", "1000")       # no more chain CTAs than slices to run
-    assert gdn.prefill_plan(1, 4096, 16, sm_count=148) == (64, 32, 1)
-    monkeypatch.setenv("GDN_TC_SLICE", "48")      # not a slice width: the model's choice stays
-    monkeypatch.delenv("GDN_PC_NC")
-    assert gdn.prefill_plan(1, 4096, 16, sm_count=148) == (32, 64, 1)
+def test_prefill_plan_applies_and_clamps_a_requested_plan():
+    plan = lambda req: gdn.prefill_plan(1, 4096, 16, sm_count=148, requested=req)
+    assert plan((64, 7)) == (64, 6, 6)           # rounded down to whole chains of 2 slices
+    assert plan((64, 1000)) == (64, 32, 1)       # no more chain CTAs than slices to run
+    assert plan((0, 0)) == plan(None) == (32, 64, 1)
+    assert plan((128, 0)) == (128, 16, 1)        # another width keeps the model's 16 chains per round
+    assert plan((0, 8)) == (32, 8, 8)            # a count alone keeps the model's width
+    assert gdn.prefill_plan(1, 81920, 32, sm_count=148, requested=(32, 500)) == (32, 128, 1)   # 74 positions max
+    for bad in ((48, 0), (0, -1)):                # not a slice width; a negative count
+        with pytest.raises(gdn.GdnError) as e:
+            plan(bad)
+        assert e.value.status == gdn.GDN_ERR_INVALID_ARG
 
 
-def test_prefill_plan_rejects_what_the_kernel_does_not_run(lib, monkeypatch):
-    monkeypatch.delenv("GDN_TC_SLICE", raising=False)
-    monkeypatch.delenv("GDN_PC_NC", raising=False)
+def test_concurrent_prefill_plans_do_not_leak_between_threads():
+    """The plan is an argument of the call, not process state: host threads asking
+    with different plans at the same time each get their own."""
+    import threading
+    errors = []
+
+    def worker(req, want):
+        for _ in range(2000):
+            got = gdn.prefill_plan(1, 4096, 16, sm_count=148, requested=req)
+            if got != want:
+                errors.append((req, got))
+                return
+
+    cases = [((64, 6), (64, 6, 6)), ((128, 3), (128, 3, 6)), (None, (32, 64, 1)), ((32, 16), (32, 16, 4))]
+    threads = [threading.Thread(target=worker, args=c) for c in cases]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errors
+
+
+def test_prefill_ex_rejects_an_invalid_plan_before_any_launch(lib):
+    for dvp, nc in ((48, 0), (64, -2)):
+        status = lib.gdn_prefill_ex(P, P, P, P, P, None, P, 1, 64, 2, 4, 128, 128, ctypes.c_float(0.0), 0,
+                                    gdn.GDN_BF16, P, P, P, 1 << 26, ctypes.byref(gdn.GdnPlan(dvp, nc)), None)
+        assert status == gdn.GDN_ERR_INVALID_ARG
+        assert "plan" in lib.gdn_last_error().decode()
+
+
+def test_prefill_plan_rejects_what_the_kernel_does_not_run(lib):
     with pytest.raises(gdn.GdnError) as e:
         gdn.prefill_plan(1, 4096, 16, dk=64, dv=64, sm_count=148)
     assert e.value.status == gdn.GDN_ERR_UNSUPPORTED
@@ -174,5 +201,5 @@ def test_prefill_plan_rejects_what_the_kernel_does_not_run(lib, monkeypatch):
             gdn.prefill_plan(a["n_seqs"], a["total_T"], a["Hv"], sm_count=a["sm_count"])
         assert e.value.status == gdn.GDN_ERR_INVALID_ARG
     out = ctypes.c_int(0)
-    assert lib.gdn_prefill_plan(1, 4096, 16, 128, 128, gdn.GDN_BF16, 148, None, ctypes.byref(out),
+    assert lib.gdn_prefill_plan(1, 4096, 16, 128, 128, gdn.GDN_BF16, 148, None, None, ctypes.byref(out),
                                 ctypes.byref(out)) == gdn.GDN_ERR_INVALID_ARG

@@ -12,9 +12,13 @@ comparison. Two gates are applied:
     night the engine chose wrong"): max error <= 1/64 of the largest |value|
     of the reference, which is much tighter than the absolute bounds for o.
 
-Full-size workloads are compared on a sample of value heads (all tokens of
-those heads), which the oracle computes exactly like the full problem.
+Full-size workloads are compared on a sample of value heads spread over the
+whole head range (all tokens of those heads), which the oracle computes
+exactly like the full problem; at the long and varlen sizes the sampled heads
+sit at different positions of the tensor-core kernel's package ring.
 """
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 import pytest
 import torch
@@ -41,7 +45,23 @@ def _gate(name, err, ref_max, tol, rel=1 / 64):
     assert err <= rel * ref_max + 1e-7, f"{name}: max abs error {err:.3e} > 1/64 of max |ref| {ref_max:.3e}"
 
 
-def run_prefill(x, chunk=0, heads=None, state_in_device=True, alias=False):
+def oracle_prefill_heads(x, heads):
+    """The oracle's prefill on the value heads in `heads` (a list; None = all),
+    one head per thread (the oracle's C code runs outside the GIL). Heads not
+    listed stay NaN."""
+    args = (x["q"], x["k"], x["v"], x["g"], x["beta"], x["state_in"], x["cu_seqlens"])
+    if heads is None:
+        return oracle.prefill(*args)
+    with ThreadPoolExecutor(max_workers=len(heads)) as ex:
+        parts = list(ex.map(lambda h: oracle.prefill(*args, heads=(h, h + 1), n_threads=1), heads))
+    ro, rs = parts[0]
+    for h, (o_h, s_h) in zip(heads[1:], parts[1:]):
+        ro[:, h] = o_h[:, h]
+        rs[:, h] = s_h[:, h]
+    return ro, rs
+
+
+def run_prefill(x, chunk=0, heads=None, state_in_device=True, alias=False, plan=None):
     d = {kk: (vv.to(DEV) if isinstance(vv, torch.Tensor) else vv) for kk, vv in x.items()}
     T, Hv, dv = d["v"].shape
     N = d["cu_seqlens"].numel() - 1
@@ -54,18 +74,18 @@ def run_prefill(x, chunk=0, heads=None, state_in_device=True, alias=False):
         s_in = d["state_in"]
         s_out = torch.full((N, Hv, dv, dk), float("nan"), dtype=torch.float32, device=DEV)
     gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], s_in, d["cu_seqlens"], chunk=chunk,
-                o=o, state_out=s_out)
+                o=o, state_out=s_out, plan=plan)
     torch.cuda.synchronize()
     gdn.device_error()
-    ro, rs = oracle.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], x["state_in"], x["cu_seqlens"],
-                            heads=heads)
+    ro, rs = oracle_prefill_heads(x, heads)
     return o, s_out, ro, rs
 
 
-def check_prefill(x, tol_o, tol_s, chunk=0, heads=None, alias=False):
-    o, s, ro, rs = run_prefill(x, chunk=chunk, heads=heads, alias=alias)
-    sel_o = (slice(None), slice(heads[0], heads[1])) if heads else None
-    sel_s = (slice(None), slice(heads[0], heads[1])) if heads else None
+def check_prefill(x, tol_o, tol_s, chunk=0, heads=None, alias=False, plan=None):
+    """`heads`: list of value heads compared (None = every head)."""
+    o, s, ro, rs = run_prefill(x, chunk=chunk, heads=heads, alias=alias, plan=plan)
+    sel_o = (slice(None), list(heads)) if heads else None
+    sel_s = (slice(None), list(heads)) if heads else None
     eo, mo = _max_err(o, ro, sel_o)
     es, ms = _max_err(s, rs, sel_s)
     print(f"o err {eo:.3e} (max|o| {mo:.3e})  state err {es:.3e} (max|S| {ms:.3e})")
@@ -116,15 +136,32 @@ def test_decode_bf16_state_small(dtype, dk, dv):
     _gate("state", es, ms, 1e-2)
 
 
+DECODE_HEADS = [0, 13, 31]   # first, middle and last value head (q/k heads 0, 6 and 15)
+
+
+def oracle_decode_heads(x, ref, heads, state_bf16=False):
+    """One oracle decode step on the value heads in `heads` (ref updated in place
+    on those heads only); returns o with the other heads NaN."""
+    o = None
+    for h in heads:
+        o_h, ref = oracle.decode(x["q"], x["k"], x["v"], x["g"], x["beta"], ref, heads=(h, h + 1),
+                                 state_bf16=state_bf16)
+        if o is None:
+            o = o_h
+        else:
+            o[:, h] = o_h[:, h]
+    return o, ref
+
+
 def test_decode_bf16_state_workload_1000_steps_sampled_heads():
     """The decode workload (64 sequences x 32 value heads, d=128, 1000 steps)
-    with a bf16 state, on value heads 0..3. Tolerances: one bf16 ulp of the
-    largest state value is about 1.2 * 2^-8 = 4.7e-3; rounding decisions that
-    fp32 and fp64 arithmetic take differently, once in a while, leave a few
-    such ulps after 1000 decaying steps: state <= 3e-2 (about 6 ulps),
-    o <= 3e-2."""
+    with a bf16 state, on value heads 0, 13 and 31, at the workload's own
+    tolerances (o <= 2e-2 at every step, state <= 1e-2 after the last) and the
+    1/64 gate. One bf16 ulp of the largest state value is about 4.7e-3: the
+    gate allows two such ulps where fp32 and fp64 arithmetic round a value to
+    different bf16 neighbours."""
     w = workloads.workload("decode")
-    heads = (0, 4)
+    sel = (slice(None), DECODE_HEADS)
     st = workloads.decode_state(w.batch, w.Hv, w.d, std=w.state_std).to(torch.bfloat16)
     ref = st.double().numpy().copy()
     sd = st.to(DEV)
@@ -132,20 +169,20 @@ def test_decode_bf16_state_workload_1000_steps_sampled_heads():
     for step in range(w.steps):
         x = workloads.decode_step_inputs(step, w.batch, w.Hqk, w.Hv, w.d)
         o = gdn.decode(x["q"].to(DEV), x["k"].to(DEV), x["v"].to(DEV), x["g"].to(DEV), x["beta"].to(DEV), sd)
-        ro, ref = oracle.decode(x["q"], x["k"], x["v"], x["g"], x["beta"], ref, heads=heads, state_bf16=True)
-        eo, _ = _max_err(o, ro, (slice(None), slice(*heads)))
+        ro, ref = oracle_decode_heads(x, ref, DECODE_HEADS, state_bf16=True)
+        eo, mo = _max_err(o, ro, sel)
         worst_o = max(worst_o, eo)
-    es, ms = _max_err(sd, ref, (slice(None), slice(*heads)))
+        _gate(f"step {step} o", eo, mo, w.tol_o)
+    es, ms = _max_err(sd, ref, sel)
     print(f"bf16-state decode 1000 steps: worst o err {worst_o:.3e}, state err {es:.3e} (max|S| {ms:.3e})")
-    assert worst_o <= 3e-2
-    assert es <= 3e-2
+    _gate("state", es, ms, w.tol_state)
 
 
 def test_decode_workload_1000_steps_sampled_heads():
     """64 sequences x 32 value heads, d=128, 1000 consecutive steps; o checked at
-    every step and the state after the last one, on value heads 0..3."""
+    every step and the state after the last one, on value heads 0, 13 and 31."""
     w = workloads.workload("decode")
-    heads = (0, 4)
+    sel = (slice(None), DECODE_HEADS)
     state = workloads.decode_state(w.batch, w.Hv, w.d, std=w.state_std)
     ref = state.double().numpy().copy()
     sd = state.to(DEV)
@@ -153,13 +190,13 @@ def test_decode_workload_1000_steps_sampled_heads():
     for step in range(w.steps):
         x = workloads.decode_step_inputs(step, w.batch, w.Hqk, w.Hv, w.d)
         o = gdn.decode(x["q"].to(DEV), x["k"].to(DEV), x["v"].to(DEV), x["g"].to(DEV), x["beta"].to(DEV), sd)
-        ro, ref = oracle.decode(x["q"], x["k"], x["v"], x["g"], x["beta"], ref, heads=heads)
-        eo, mo = _max_err(o, ro, (slice(None), slice(*heads)))
+        ro, ref = oracle_decode_heads(x, ref, DECODE_HEADS)
+        eo, mo = _max_err(o, ro, sel)
         worst_o = max(worst_o, eo)
-        assert eo <= w.tol_o, f"step {step}: o err {eo:.3e}"
-    es, ms = _max_err(sd, ref, (slice(None), slice(*heads)))
+        _gate(f"step {step} o", eo, mo, w.tol_o)
+    es, ms = _max_err(sd, ref, sel)
     print(f"decode 1000 steps: worst o err {worst_o:.3e}, state err {es:.3e} (max|S| {ms:.3e})")
-    assert es <= w.tol_state
+    _gate("state", es, ms, w.tol_state)
     assert not torch.isnan(sd).any()
 
 
@@ -212,10 +249,12 @@ def test_prefill_workload_qwen08b_layer_full():
     check_prefill(workloads.inputs_for(w), w.tol_o, w.tol_state)
 
 
-@pytest.mark.parametrize("T", [32768, 81920])
-def test_prefill_workload_long_sampled_heads(T):
+@pytest.mark.parametrize("T,heads", [(32768, [0, 9, 18, 31]), (81920, [0, 13, 31])])
+def test_prefill_workload_long_sampled_heads(T, heads):
+    """The long prompts (16 q/k, 32 value heads) on heads spread over the range:
+    with 32 chains of 128 state rows each head runs at its own ring position."""
     w = workloads.workload("long", T=T)
-    check_prefill(workloads.inputs_for(w), w.tol_o, w.tol_state, heads=(0, 2) if T > 40000 else (0, 3))
+    check_prefill(workloads.inputs_for(w), w.tol_o, w.tol_state, heads=heads)
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
@@ -241,26 +280,22 @@ def test_prefill_many_short_sequences_many_rounds():
 
 
 @pytest.mark.parametrize("dvp,nc", [(32, 0), (64, 0), (128, 0), (64, 6), (128, 3)])
-def test_prefill_every_slice_width_and_split(dvp, nc, monkeypatch):
+def test_prefill_every_slice_width_and_split(dvp, nc):
     """The tensor-core kernel with each state-slice width, and with so few
-    state-carrying CTAs that the chains run in several rounds; the result must
-    not change beyond rounding."""
-    monkeypatch.setenv("GDN_TC_SLICE", str(dvp))
-    if nc:
-        monkeypatch.setenv("GDN_PC_NC", str(nc))
+    state-carrying CTAs that the chains run in several rounds (an explicit
+    launch plan; nc = 0 keeps the model's CTA count); the result must not
+    change beyond rounding."""
     x = workloads.prefill_inputs([300, 129, 64, 1], Hqk=4, Hv=8, d=128, seed=909 + dvp, state_std=0.05)
-    check_prefill(x, 2e-2, 1e-2)
+    check_prefill(x, 2e-2, 1e-2, plan=(dvp, nc))
 
 
 @pytest.mark.parametrize("dvp,nc", [(32, 4), (64, 2), (64, 4), (128, 2)])
-def test_prefill_long_chains_in_several_rounds(dvp, nc, monkeypatch):
+def test_prefill_long_chains_in_several_rounds(dvp, nc):
     """Chains far longer than the package ring (2500 tokens: 40 chunks, the ring
     wraps three times per chain) run in two to four rounds: every ring slot is
     reused many times within a round and across the round boundary."""
-    monkeypatch.setenv("GDN_TC_SLICE", str(dvp))
-    monkeypatch.setenv("GDN_PC_NC", str(nc))
     x = workloads.prefill_inputs([2500], Hqk=2, Hv=4, d=128, seed=5150 + dvp + nc, state_std=0.05)
-    check_prefill(x, 2e-2, 1e-2)
+    check_prefill(x, 2e-2, 1e-2, plan=(dvp, nc))
 
 
 def test_prefill_on_a_side_stream_into_caller_buffers():
@@ -288,5 +323,7 @@ def test_prefill_on_a_side_stream_into_caller_buffers():
 
 
 def test_prefill_workload_varlen_sampled_heads():
+    """8 packed sequences of 128..8192 tokens, 32 value heads, per-sequence
+    states: value heads 0, 9, 18 and 31 of every sequence."""
     w = workloads.workload("varlen")
-    check_prefill(workloads.inputs_for(w), w.tol_o, w.tol_state, heads=(0, 4))
+    check_prefill(workloads.inputs_for(w), w.tol_o, w.tol_state, heads=[0, 9, 18, 31])

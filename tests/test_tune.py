@@ -40,21 +40,6 @@ def test_gate_rejects_unwritten_and_distant_outputs():
     assert tune.gate(torch.empty(0, 8), torch.empty(0, 8))[0]
 
 
-def test_plan_override_sets_and_restores_the_environment(monkeypatch):
-    monkeypatch.setenv("GDN_TC_SLICE", "128")
-    monkeypatch.delenv("GDN_PC_NC", raising=False)
-    with tune.plan_override(64, 32):
-        assert os.environ["GDN_TC_SLICE"] == "64" and os.environ["GDN_PC_NC"] == "32"
-    assert os.environ["GDN_TC_SLICE"] == "128" and "GDN_PC_NC" not in os.environ
-    with tune.plan_override(None, None):   # the library's own choice: both unset
-        assert "GDN_TC_SLICE" not in os.environ and "GDN_PC_NC" not in os.environ
-    assert os.environ["GDN_TC_SLICE"] == "128"
-    with pytest.raises(KeyError):
-        with tune.plan_override(32, 8):
-            raise KeyError("inside")
-    assert os.environ["GDN_TC_SLICE"] == "128" and "GDN_PC_NC" not in os.environ
-
-
 def test_check_problem_has_a_full_and_a_partial_chunk_and_a_state():
     q, k, v, g, beta, s, cu = tune.check_problem(2, 4, 128, 128, torch.bfloat16, "cpu")
     assert q.shape == (101, 2, 128) and v.shape == (101, 4, 128) and q.dtype == torch.bfloat16
@@ -147,14 +132,15 @@ def test_tune_refuses_shapes_without_launch_plans():
 
 def test_device_runner_applies_the_plan_times_and_fills_fresh_outputs(monkeypatch):
     """The device leg's own lines, with the library call, the error check and the
-    CUDA events replaced by stand-ins (no GPU): the plan is in force for every
-    call and undone after, the gated outputs come from a call into NaN-filled
+    CUDA events replaced by stand-ins (no GPU): the plan is passed to every
+    call (no process state), the gated outputs come from a call into NaN-filled
     buffers, and the time is the events' over the timed calls."""
     import gated_deltanet_linear_21_b200 as pkg
     seen = []
 
-    def fake_prefill(q, k, v, g, beta, state_in=None, cu_seqlens=None, *, o=None, state_out=None, **kw):
-        seen.append((os.environ.get("GDN_TC_SLICE"), os.environ.get("GDN_PC_NC"), o is not None))
+    def fake_prefill(q, k, v, g, beta, state_in=None, cu_seqlens=None, *, o=None, state_out=None, plan=None,
+                     **kw):
+        seen.append((plan, o is not None))
         T, Hv, dv = v.shape
         N = cu_seqlens.numel() - 1
         if o is not None:
@@ -178,19 +164,16 @@ def test_device_runner_applies_the_plan_times_and_fills_fresh_outputs(monkeypatc
     monkeypatch.setattr(pkg, "device_error", lambda stream=None: None)
     monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
     monkeypatch.setattr(torch.cuda, "Event", FakeEvent)
-    monkeypatch.delenv("GDN_TC_SLICE", raising=False)
-    monkeypatch.setenv("GDN_PC_NC", "5")
     q, k, v, g, beta = _fake_problem()
     cu = torch.tensor([0, 130], dtype=torch.int32)
     o, s, ms = tune._device_runner((q, k, v, g, beta, None, cu), (64, 32), 3)
     assert ms == pytest.approx(2.0)                                   # 6 ms over 3 timed calls
     assert o.dtype == torch.bfloat16 and o.shape == v.shape and torch.equal(o.float(), (v.float() * 2).to(o.dtype).float())
     assert s.shape == (1, 4, 128, 128) and bool((s == 3.0).all())
-    assert seen == [("64", "32", False)] * 4 + [("64", "32", True)]  # warm-up, 3 timed, the gated call
-    assert "GDN_TC_SLICE" not in os.environ and os.environ["GDN_PC_NC"] == "5"
+    assert seen == [((64, 32), False)] * 4 + [((64, 32), True)]  # warm-up, 3 timed, the gated call
     seen.clear()
     o, s, ms = tune._device_runner((q, k, v, g, beta, None, cu), None, 0)   # the default plan, untimed
-    assert math.isnan(ms) and seen == [(None, None, True)]
+    assert math.isnan(ms) and seen == [(None, True)]
     # and the whole selection through the device leg
     best, results = tune.tune_prefill(q, k, v, g, beta, None, cu, plans=[(32, 16), (128, 4)], reps=2)
     assert all(r.ok for r in results) and (best.dvp, best.nc) == (32, 16)

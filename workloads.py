@@ -99,6 +99,19 @@ def _gates(gen: torch.Generator, shape):
     return g, beta
 
 
+def log_sigmoid_gates(gen: torch.Generator, shape, mean: float, std: float):
+    """g = log sigmoid(x), x ~ N(mean, std^2) drawn in fp64, rounded once to fp32
+    (mean 3, std 1 is the workloads' own decay; negative means decay strongly)."""
+    x = torch.randn(shape, generator=gen, dtype=torch.float64) * std + mean
+    return torch.nn.functional.logsigmoid(x).to(torch.float32)
+
+
+def shifted_log_decay(gen: torch.Generator, shape, mean: float, std: float):
+    """g ~ N(mean, std^2) drawn in fp64, rounded once to fp32 (no sigmoid: with a
+    mean of -5 every token decays the state by about e^-5)."""
+    return (torch.randn(shape, generator=gen, dtype=torch.float64) * std + mean).to(torch.float32)
+
+
 def prefill_inputs(lengths, Hqk, Hv, d, dtype=torch.bfloat16, seed=SEED_TOKENS + 1,
                    state_std=0.0, state_seed=None, dv=None):
     """Packed prefill inputs on the CPU.
