@@ -113,7 +113,8 @@ def traffic_record(kernel):
 
 class ClockSampler:
     """Samples the SM clock and the clock-event (throttle) reasons through NVML
-    every ~2 ms while a timed region runs (reading only; nothing is changed)."""
+    about every 0.5 ms while a timed region runs (reading only; nothing is
+    changed)."""
 
     REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
                ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
@@ -155,7 +156,7 @@ class ClockSampler:
                     self.samples.append((mhz, rs))
                 except Exception:
                     pass
-                self._stop.wait(0.002)
+                self._stop.wait(0.0005)
 
         self._thread = threading.Thread(target=loop, daemon=True)
         self._thread.start()
@@ -207,14 +208,36 @@ def timed(fn, stream):
     return a.elapsed_time(b)
 
 
+MIN_SAMPLED_MS = 300.0
+
+
+def timed_replays(graph, stream, steps, sampler=None, min_ms=MIN_SAMPLED_MS):
+    """Per-step device time of a graph holding `steps` steps: each replay is timed
+    on its own with CUDA events (exactly `steps` steps between the events), and
+    the replays are repeated until about `min_ms` of device time has passed (at
+    least 5), so that the clock sampler sees the whole region many times; the
+    median replay is returned with the number of replays."""
+    first = timed(graph.replay, stream)
+    reps = max(5, min(2000, int(min_ms / max(first, 1e-3)) + 1))
+    times = []
+    if sampler is not None:
+        with sampler:
+            for _ in range(reps):
+                times.append(timed(graph.replay, stream))
+    else:
+        for _ in range(reps):
+            times.append(timed(graph.replay, stream))
+    return statistics.median(times) / steps, reps
+
+
 # ------------------------------------------------------------ our workload ---
-def device_prefill_inputs(lengths, Hqk, Hv, d, seed, device, state_std=0.0):
+def device_prefill_inputs(lengths, Hqk, Hv, d, seed, device, state_std=0.0, dtype=torch.bfloat16):
     """Seeded inputs generated on the device (same distributions as workloads.py)."""
     gen = torch.Generator(device=device).manual_seed(seed)
     T = sum(lengths)
-    q = torch.randn(T, Hqk, d, generator=gen, device=device).to(torch.bfloat16)
-    k = torch.randn(T, Hqk, d, generator=gen, device=device).to(torch.bfloat16)
-    v = torch.randn(T, Hv, d, generator=gen, device=device).to(torch.bfloat16)
+    q = torch.randn(T, Hqk, d, generator=gen, device=device).to(dtype)
+    k = torch.randn(T, Hqk, d, generator=gen, device=device).to(dtype)
+    v = torch.randn(T, Hv, d, generator=gen, device=device).to(dtype)
     x = torch.randn(T, Hv, generator=gen, device=device, dtype=torch.float64) + 3.0
     y = torch.randn(T, Hv, generator=gen, device=device, dtype=torch.float64)
     g = torch.nn.functional.logsigmoid(x).float()
@@ -227,14 +250,14 @@ def device_prefill_inputs(lengths, Hqk, Hv, d, seed, device, state_std=0.0):
     return dict(q=q, k=k, v=v, g=g, beta=beta, cu_seqlens=cu.to(device), state_in=s0)
 
 
-def run_prefill_bench(gdn, w, steps, warmup, device, rank, sampler=None):
+def run_prefill_bench(gdn, w, steps, warmup, device, rank, sampler=None, min_ms=MIN_SAMPLED_MS):
     stream = torch.cuda.current_stream()
     T = w.total_tokens
     one = prefill_bytes(T, w.Hqk, w.Hv, w.d, len(w.lengths), w.state_std > 0)
-    copies = max(2, -(-3 * L2_BYTES // one))   # rotate inputs over > 3x L2
+    copies = l2_copies(w)   # rotate inputs over > 3x L2
     bufs = [device_prefill_inputs(w.lengths, w.Hqk, w.Hv, w.d, 7919 * rank + 31 * i + w.index,
-                                  device, w.state_std) for i in range(copies)]
-    outs = [(torch.empty(T, w.Hv, w.d, dtype=torch.bfloat16, device=device),
+                                  device, w.state_std, w.torch_dtype) for i in range(copies)]
+    outs = [(torch.empty(T, w.Hv, w.d, dtype=w.torch_dtype, device=device),
              torch.empty(len(w.lengths), w.Hv, w.d, w.d, device=device)) for _ in range(copies)]
 
     def step(i):
@@ -254,15 +277,12 @@ def run_prefill_bench(gdn, w, steps, warmup, device, rank, sampler=None):
     torch.cuda.synchronize()
     graph.replay()   # untimed replay: first-replay costs
     torch.cuda.synchronize()
-    if sampler is not None:
-        with sampler:
-            ms = timed(graph.replay, stream) / steps
-    else:
-        ms = timed(graph.replay, stream) / steps
-    return dict(ms=ms, tokens=T, bytes=one, copies=copies, graph=graph)
+    ms, reps = timed_replays(graph, stream, steps, sampler, min_ms=min_ms)
+    return dict(ms=ms, tokens=T, bytes=one, copies=copies, graph=graph, replays=reps)
 
 
-def run_decode_bench(gdn, w, steps_timed, warmup, device, rank, sampler=None, state_dtype=torch.float32):
+def run_decode_bench(gdn, w, steps_timed, warmup, device, rank, sampler=None, state_dtype=torch.float32,
+                     min_ms=MIN_SAMPLED_MS):
     stream = torch.cuda.current_stream()
     B, Hqk, Hv, d = w.batch, w.Hqk, w.Hv, w.d
     gen = torch.Generator(device=device).manual_seed(workloads.SEED_DECODE_STEP + 7919 * rank)
@@ -286,12 +306,8 @@ def run_decode_bench(gdn, w, steps_timed, warmup, device, rank, sampler=None, st
         run(0, n)
     graph.replay()
     torch.cuda.synchronize()
-    if sampler is not None:
-        with sampler:
-            ms = timed(graph.replay, stream) / n
-    else:
-        ms = timed(graph.replay, stream) / n
-    return dict(ms=ms, bytes=decode_bytes(B, Hqk, Hv, d, state.element_size()), steps=n)
+    ms, reps = timed_replays(graph, stream, n, sampler, min_ms=min_ms)
+    return dict(ms=ms, bytes=decode_bytes(B, Hqk, Hv, d, state.element_size()), steps=n, replays=reps)
 
 
 def run_e2e(gdn, w, steps, device):
@@ -356,24 +372,74 @@ def run_e2e(gdn, w, steps, device):
     return dict(ms=ms, h2d=h2d, d2h=d2h, tokens=T)
 
 
-def cpu_baseline(w, budget_s=10.0):
-    """The fp64 oracle as it stands, on the host cores, over whole copies of the
-    workload until about budget_s seconds have passed."""
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def host_read_gbs(nbytes=1 << 30, passes=5):
+    """Host sequential-read bandwidth: every core sums its own slice of a 1 GiB
+    fp64 array (numpy releases the GIL inside the reduction); best of several
+    passes, after a pass that touches every page."""
+    import threading
+
+    import numpy as np
+    a = np.ones(nbytes // 8)
+    cores = os.cpu_count() or 1
+    parts = np.array_split(a, cores)
+    best = 0.0
+    for _ in range(passes + 1):
+        ts = [threading.Thread(target=np.add.reduce, args=(p,)) for p in parts]
+        t0 = time.perf_counter()
+        for t in ts:
+            t.start()
+        for t in ts:
+            t.join()
+        best = max(best, a.nbytes / (time.perf_counter() - t0) / 1e9)
+    return round(best, 1), cores
+
+
+def cpu_baseline(w, reps=3):
+    """The fp64 oracle as it stands, on the host cores: median of `reps` whole
+    passes of the workload with every core (OpenMP over (sequence, head)) and
+    with one core, next to the host CPU model and its read bandwidth."""
     import oracle
     x = workloads.inputs_for(w)
     cores = os.cpu_count() or 1
-    t0 = time.perf_counter()
-    reps = 0
-    while True:
-        oracle.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], x["state_in"], x["cu_seqlens"],
-                       n_threads=cores)
-        reps += 1
-        el = time.perf_counter() - t0
-        if el >= budget_s or reps >= 50:
-            break
-    return dict(value=reps * w.total_tokens / el, unit="tokens/s", cores=cores, kind="oracle",
-                sample=f"{reps} full pass(es) of the workload ({w.total_tokens} tokens x {w.Hv} heads), "
-                       f"{el:.1f} s wall")
+
+    def median_pass(threads):
+        times = []
+        for _ in range(reps):
+            t0 = time.perf_counter()
+            oracle.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], x["state_in"], x["cu_seqlens"],
+                           n_threads=threads)
+            times.append(time.perf_counter() - t0)
+        return statistics.median(times)
+
+    t_all = median_pass(cores)
+    t_one = median_pass(1)
+    gbs, bw_threads = host_read_gbs()
+    return dict(value=w.total_tokens / t_all, unit="tokens/s", cores=cores, kind="oracle",
+                sample=f"median of {reps} full passes of the workload ({w.total_tokens} tokens x {w.Hv} heads) "
+                       f"with {cores} threads: {t_all:.3f} s each",
+                single_core={"value": w.total_tokens / t_one, "unit": "tokens/s", "cores": 1,
+                             "sample": f"median of {reps} full passes with 1 thread: {t_one:.2f} s each"},
+                cpu_model=cpu_model(),
+                host_read_gbs={"value": gbs, "threads": bw_threads,
+                               "method": "every core sums its slice of a 1 GiB fp64 array, best of 5 passes"})
+
+
+def l2_copies(w):
+    """Copies of a prefill workload's inputs the GPU arm rotates over between
+    timed calls, so that they span more than 3x the 126 MB L2."""
+    one = prefill_bytes(w.total_tokens, w.Hqk, w.Hv, w.d, len(w.lengths), w.state_std > 0)
+    return max(2, -(-3 * L2_BYTES // one))
 
 
 def workload_config(w, copies=None, n=1):
@@ -389,8 +455,19 @@ def workload_config(w, copies=None, n=1):
            "global_batch": len(w.lengths) * n, "seq_len": w.total_tokens,
            "parallelism": f"dp{n} (independent sequences per rank, no exchange)"}
     if copies:
-        cfg["l2"] = f"inputs rotated over {copies} copies (> 3x the 126 MB L2)"
+        cfg["l2"] = f"GPU arm: inputs rotated over {copies} copies (> 3x the 126 MB L2)"
     return cfg
+
+
+def prefill_subline(r, w, steps, ms_max, world, pk, pk_kind):
+    """A prefill workload's sub-object of the JSON line."""
+    fl = prefill_flops_per_token_head(w.chunk, w.d) * r["tokens"] * w.Hv
+    return {"value": aggregate_rate(r["tokens"], ms_max, world), "unit": "tokens/s", "ms_per_step": ms_max,
+            "steps": steps, "timed_replays": r["replays"], "gpu_launches": steps,
+            "config": workload_config(w, r["copies"], world),
+            "roofline": roofline_tensor(fl, r["ms"], pk, pk_kind),
+            "roofline_hbm_view": roofline_hbm(r["bytes"], r["ms"], pk, pk_kind),
+            "binding_frac": binding_frac(fl, r["bytes"], r["ms"], pk)}
 
 
 def roofline_tensor(flops, ms, pk, kind, key="bf16_tflops", traffic=None):
@@ -467,7 +544,7 @@ def main():
         line = {"impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": args.gpus,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": DATA,
-                "config": workload_config(w),
+                "config": workload_config(w, l2_copies(w) if w.kind == "prefill" else None),
                 "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
                                  "sample": sample},
                 "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -511,6 +588,7 @@ def main():
                                             traffic=tr["bytes_per_launch"] if tr else None),
                 "roofline_hbm_view": roofline_hbm(r["bytes"], r["ms"], pk, pk_kind),
                 "binding_frac": binding_frac(flops, r["bytes"], r["ms"], pk),
+                "timed_replays": r["replays"],
                 "gpu_launches": args.steps, "clocks": clk.summary()}
         del r["graph"]
     else:
@@ -563,12 +641,24 @@ def main():
         del rl["graph"]
         msl = max_over_ranks(rl["ms"])
         fl = prefill_flops_per_token_head(wl.chunk, wl.d) * rl["tokens"] * wl.Hv
-        line["long_prefill"] = {"value": aggregate_rate(rl["tokens"], msl, world), "unit": "tokens/s",
-                                "ms_per_step": msl, "steps": nl, "gpu_launches": nl,
-                                "config": workload_config(wl, rl["copies"], world),
-                                "roofline": roofline_tensor(fl, rl["ms"], pk, pk_kind),
-                                "roofline_hbm_view": roofline_hbm(rl["bytes"], rl["ms"], pk, pk_kind),
-                                "binding_frac": binding_frac(fl, rl["bytes"], rl["ms"], pk)}
+        line["long_prefill"] = prefill_subline(rl, wl, nl, msl, world, pk, pk_kind)
+        # the longest prompt: 81920 tokens, 16 q/k and 32 v heads
+        wx = workloads.workload("long", T=81920)
+        nx = max(2, args.steps // 10)
+        rx = run_prefill_bench(gdn, wx, nx, args.warmup, device, rank)
+        del rx["graph"]
+        line["long_prefill_81920"] = prefill_subline(rx, wx, nx, max_over_ranks(rx["ms"]), world, pk, pk_kind)
+        # packed varlen: 8 sequences of 128..8192 tokens with their own states
+        wv = workloads.workload("varlen")
+        nv = max(2, args.steps // 4)
+        rv = run_prefill_bench(gdn, wv, nv, args.warmup, device, rank)
+        del rv["graph"]
+        line["varlen_prefill"] = prefill_subline(rv, wv, nv, max_over_ranks(rv["ms"]), world, pk, pk_kind)
+        # the 4096-token layer with f16 inputs and output
+        wf = workloads.workload("prefill", dtype="f16")
+        rf = run_prefill_bench(gdn, wf, args.steps, args.warmup, device, rank)
+        del rf["graph"]
+        line["prefill_f16"] = prefill_subline(rf, wf, args.steps, max_over_ranks(rf["ms"]), world, pk, pk_kind)
 
     if w.kind == "prefill":
         e = run_e2e(gdn, w, max(3, args.steps // 2), device)

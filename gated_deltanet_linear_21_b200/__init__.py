@@ -22,15 +22,17 @@ import torch
 __all__ = ["prefill", "prefill_noalloc", "decode", "prefill_workspace_bytes", "prefill_plan", "device_error",
            "wait_selftest",
            "GdnError",
-           "lib", "library_path", "GDN_BF16", "GDN_F32", "GDN_F16"]
+           "lib", "debug_lib", "library_path", "debug_library_path", "GDN_BF16", "GDN_F32", "GDN_F16"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_PKG, "libgdn.so")
+debug_library_path = os.path.join(_PKG, "libgdn_debug.so")   # GDN_DEBUG build: device-side index checks
 
-GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_DEVICE_TIMEOUT = range(5)
+(GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_DEVICE_TIMEOUT,
+ GDN_ERR_DEVICE_CHECK) = range(6)
 GDN_BF16, GDN_F32, GDN_F16 = 0, 1, 2
 STATUS_NAMES = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED",
-                3: "GDN_ERR_CUDA", 4: "GDN_ERR_DEVICE_TIMEOUT"}
+                3: "GDN_ERR_CUDA", 4: "GDN_ERR_DEVICE_TIMEOUT", 5: "GDN_ERR_DEVICE_CHECK"}
 
 
 class GdnPlan(ctypes.Structure):
@@ -74,7 +76,20 @@ SIGNATURES = {
     "gdn_prefill_ex": (_i, [_vp, _vp, _vp, _fp, _fp, _fp, _i32p, _i, _i64, _i, _i, _i, _i, _f, _i, _i,
                             _vp, _fp, _vp, _sz, _vp, _vp]),
     "gdn_prefill_plan": (_i, [_i, _i64, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
+    "gdn_debug_checks": (_i, []),
 }
+
+
+def _open(path):
+    if not os.path.exists(path):
+        raise ImportError(
+            f"{path} is missing: build it with "
+            "`python -m gated_deltanet_linear_21_b200.build` (there is no CPU fallback)")
+    handle = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(handle, name)
+        fn.restype, fn.argtypes = res, args
+    return handle
 
 
 def lib():
@@ -82,16 +97,22 @@ def lib():
     global _lib
     with _lock:
         if _lib is None:
-            if not os.path.exists(library_path):
-                raise ImportError(
-                    f"{library_path} is missing: build it with "
-                    "`python -m gated_deltanet_linear_21_b200.build` (there is no CPU fallback)")
-            handle = ctypes.CDLL(library_path)
-            for name, (res, args) in SIGNATURES.items():
-                fn = getattr(handle, name)
-                fn.restype, fn.argtypes = res, args
-            _lib = handle
+            _lib = _open(library_path)
     return _lib
+
+
+_debug_lib = None
+
+
+def debug_lib():
+    """Load libgdn_debug.so, the GDN_DEBUG build (same C ABI, device-side index
+    checks reported as GDN_ERR_DEVICE_CHECK by its gdn_device_error); a ctypes
+    handle for direct calls. The Python wrappers above always use libgdn.so."""
+    global _debug_lib
+    with _lock:
+        if _debug_lib is None:
+            _debug_lib = _open(debug_library_path)
+    return _debug_lib
 
 
 def _check(status: int):

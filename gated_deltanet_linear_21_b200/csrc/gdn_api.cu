@@ -41,6 +41,7 @@ gdn_status ok() {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 bool head_dim_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+bool dtype_ok(gdn_dtype dtype) { return dtype == GDN_BF16 || dtype == GDN_F32 || dtype == GDN_F16; }
 
 // Allow a kernel the full opt-in shared memory, once per (kernel, device), so
 // that later calls (including ones inside CUDA-graph capture) only launch.
@@ -103,7 +104,7 @@ gdn_status check_decode(const char* fn, const void* q, const void* k, const void
     return fail(GDN_ERR_INVALID_ARG, "%s: Hv=%d must be a positive multiple of Hqk=%d", fn, Hv, Hqk);
   if (!head_dim_ok(dk) || !head_dim_ok(dv))
     return fail(GDN_ERR_UNSUPPORTED, "%s: dk=%d, dv=%d (supported: 16, 32, 64, 128)", fn, dk, dv);
-  if (dtype != GDN_BF16 && dtype != GDN_F32) return fail(GDN_ERR_INVALID_ARG, "%s: unknown dtype %d", fn, (int)dtype);
+  if (!dtype_ok(dtype)) return fail(GDN_ERR_INVALID_ARG, "%s: unknown dtype %d", fn, (int)dtype);
   if ((int64_t)B * Hv > 0x7fffffff) return fail(GDN_ERR_INVALID_ARG, "%s: B*Hv too large", fn);
   if (B == 0) {
     *done = true;
@@ -163,8 +164,9 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 3-D bf16 map over a token-major [T][H][D] tensor: dims (D, H, T), box (box_d, 1, 64).
-bool make_map(CUtensorMap* m, const void* base, int D, int H, int T, int box_d) {
+// 3-D map of 16-bit elements (bf16 or f16) over a token-major [T][H][D] tensor:
+// dims (D, H, T), box (box_d, 1, 64).
+bool make_map(CUtensorMap* m, const void* base, int D, int H, int T, int box_d, CUtensorMapDataType type) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T};
@@ -175,7 +177,7 @@ bool make_map(CUtensorMap* m, const void* base, int D, int H, int T, int box_d) 
   CUtensorMapSwizzle sw = row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                           : row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
                                             : CU_TENSOR_MAP_SWIZZLE_32B;
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = enc(m, type, 3, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -204,13 +206,14 @@ __global__ void wait_selftest_kernel(long long max_cycles) {
 }
 
 bool uses_pc_prefill(gdn_dtype dtype, int dk, int dv) {
-  return dtype == GDN_BF16 && dk == 128 && dv == 128;
+  return (dtype == GDN_BF16 || dtype == GDN_F16) && dk == 128 && dv == 128;
 }
 
-template <int DVP>
+
+template <int DVP, typename T>
 gdn_status launch_pc(const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& om,
                      const gdn::pc::Params& prm, int grid, cudaStream_t st) {
-  auto kern = gdn::pc::prefill_pc_kernel<DVP>;
+  auto kern = gdn::pc::prefill_pc_kernel<DVP, T>;
   if (gdn_status s = allow_smem(kern, "gdn_prefill")) return s;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
@@ -302,8 +305,8 @@ PcLaunchPlan resolve_pc(long chains, int64_t total_T, int n_seqs, int Hv, int sm
 
 gdn_status launch_prefill_pc(const void* q, const void* k, const void* v, const float* g, const float* beta,
                              const float* state_in, const int32_t* cu, int n_seqs, int64_t total_T, int Hqk,
-                             int Hv, float scale, void* o, float* state_out, void* ws, const gdn_plan* req,
-                             cudaStream_t st) {
+                             int Hv, float scale, gdn_dtype dtype, void* o, float* state_out, void* ws,
+                             const gdn_plan* req, cudaStream_t st) {
   const long chains = (long)n_seqs * Hv;
   const int sms = sm_count();
   if (sms < 16) return fail(GDN_ERR_CUDA, "gdn_prefill: cannot query the multiprocessor count");
@@ -313,9 +316,10 @@ gdn_status launch_prefill_pc(const void* q, const void* k, const void* v, const 
   if (lp.rounds > gdn::pc::kMaxRounds)
     return fail(GDN_ERR_UNSUPPORTED, "gdn_prefill: %ld sequence-heads is more than this kernel schedules", chains);
   CUtensorMap qm, km, vm, om;
-  if (!make_map(&qm, q, 128, Hqk, (int)total_T, 64) || !make_map(&km, k, 128, Hqk, (int)total_T, 64) ||
-      !make_map(&vm, v, 128, Hv, (int)total_T, std::min(dvp, 64)) ||
-      !make_map(&om, o, 128, Hv, (int)total_T, std::min(dvp, 64)))
+  const CUtensorMapDataType ty = dtype == GDN_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (!make_map(&qm, q, 128, Hqk, (int)total_T, 64, ty) || !make_map(&km, k, 128, Hqk, (int)total_T, 64, ty) ||
+      !make_map(&vm, v, 128, Hv, (int)total_T, std::min(dvp, 64), ty) ||
+      !make_map(&om, o, 128, Hv, (int)total_T, std::min(dvp, 64), ty))
     return fail(GDN_ERR_CUDA, "gdn_prefill: cuTensorMapEncodeTiled unavailable or failed");
   cudaError_t e = cudaMemsetAsync(ws, 0, gdn::pc::Workspace::zeroed_bytes(nc / slices), st);
   if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "gdn_prefill: %s", cudaGetErrorString(e));
@@ -324,7 +328,7 @@ gdn_status launch_prefill_pc(const void* q, const void* k, const void* v, const 
   prm.beta = beta;
   prm.state_in = state_in;
   prm.cu_seqlens = cu;
-  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.o = o;
   prm.state_out = state_out;
   prm.ws = static_cast<uint8_t*>(ws);
   prm.n_seqs = n_seqs;
@@ -333,16 +337,21 @@ gdn_status launch_prefill_pc(const void* q, const void* k, const void* v, const 
   prm.total_T = (int)total_T;
   prm.scale = scale;
   prm.n_chain_ctas = (int)nc;
-  if (dvp == 32) return launch_pc<32>(qm, km, vm, om, prm, sms, st);
-  if (dvp == 64) return launch_pc<64>(qm, km, vm, om, prm, sms, st);
-  return launch_pc<128>(qm, km, vm, om, prm, sms, st);
+  if (dtype == GDN_F16) {
+    if (dvp == 32) return launch_pc<32, __half>(qm, km, vm, om, prm, sms, st);
+    if (dvp == 64) return launch_pc<64, __half>(qm, km, vm, om, prm, sms, st);
+    return launch_pc<128, __half>(qm, km, vm, om, prm, sms, st);
+  }
+  if (dvp == 32) return launch_pc<32, __nv_bfloat16>(qm, km, vm, om, prm, sms, st);
+  if (dvp == 64) return launch_pc<64, __nv_bfloat16>(qm, km, vm, om, prm, sms, st);
+  return launch_pc<128, __nv_bfloat16>(qm, km, vm, om, prm, sms, st);
 }
 
 }  // namespace
 
 extern "C" {
 
-int gdn_version(void) { return (0 << 16) | 3; }
+int gdn_version(void) { return (0 << 16) | 4; }
 
 const char* gdn_last_error(void) { return t_last_error.c_str(); }
 
@@ -362,7 +371,7 @@ gdn_status gdn_prefill_plan(int n_seqs, int64_t total_T, int Hv, int dk, int dv,
     return fail(GDN_ERR_INVALID_ARG, "gdn_prefill_plan: n_seqs %d, Hv %d, total_T %lld", n_seqs, Hv,
                 (long long)total_T);
   if (!uses_pc_prefill(dtype, dk, dv))
-    return fail(GDN_ERR_UNSUPPORTED, "gdn_prefill_plan: the tensor-core kernel takes bf16 with dk = dv = 128");
+    return fail(GDN_ERR_UNSUPPORTED, "gdn_prefill_plan: the tensor-core kernel takes bf16 or f16 with dk = dv = 128");
   const int sms = sm_count_arg > 0 ? sm_count_arg : sm_count();
   if (sms < 16) return fail(GDN_ERR_INVALID_ARG, "gdn_prefill_plan: %d multiprocessors", sms);
   const PcLaunchPlan lp = resolve_pc((long)n_seqs * Hv, total_T, n_seqs, Hv, sms, requested);
@@ -387,8 +396,7 @@ gdn_status gdn_prefill_ex(const void* q, const void* k, const void* v, const flo
     return fail(GDN_ERR_INVALID_ARG, "gdn_prefill: Hv=%d must be a positive multiple of Hqk=%d", Hv, Hqk);
   if (!head_dim_ok(dk) || !head_dim_ok(dv))
     return fail(GDN_ERR_UNSUPPORTED, "gdn_prefill: dk=%d, dv=%d (supported: 16, 32, 64, 128)", dk, dv);
-  if (dtype != GDN_BF16 && dtype != GDN_F32)
-    return fail(GDN_ERR_INVALID_ARG, "gdn_prefill: unknown dtype %d", (int)dtype);
+  if (!dtype_ok(dtype)) return fail(GDN_ERR_INVALID_ARG, "gdn_prefill: unknown dtype %d", (int)dtype);
   if (n_seqs == 0) return ok();
   if (!cu_seqlens || !state_out)
     return fail(GDN_ERR_INVALID_ARG, "gdn_prefill: cu_seqlens and state_out must not be NULL");
@@ -401,7 +409,7 @@ gdn_status gdn_prefill_ex(const void* q, const void* k, const void* v, const flo
     return fail(GDN_ERR_INVALID_ARG, "gdn_prefill: g, beta and cu_seqlens must be 4-byte aligned");
   if (scale <= 0.f) scale = 1.0f / sqrtf((float)dk);
   int C = chunk;
-  if (C == 0) C = (dtype == GDN_BF16 && dk == 128 && dv == 128) ? 64 : 16;
+  if (C == 0) C = uses_pc_prefill(dtype, dk, dv) ? 64 : 16;
   if (C != 16 && C != 32 && C != 64)
     return fail(GDN_ERR_UNSUPPORTED, "gdn_prefill: chunk=%d (supported: 16, 32, 64)", C);
   const size_t need = gdn_prefill_workspace_bytes(n_seqs, Hv, dk, dv, dtype);
@@ -410,11 +418,14 @@ gdn_status gdn_prefill_ex(const void* q, const void* k, const void* v, const flo
                 need, workspace_bytes);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (uses_pc_prefill(dtype, dk, dv) && C == 64 && total_T > 0)
-    return launch_prefill_pc(q, k, v, g, beta, state_in, cu_seqlens, n_seqs, total_T, Hqk, Hv, scale, o, state_out,
-                             workspace, plan, st);
+    return launch_prefill_pc(q, k, v, g, beta, state_in, cu_seqlens, n_seqs, total_T, Hqk, Hv, scale, dtype, o,
+                             state_out, workspace, plan, st);
   if (dtype == GDN_F32)
     return launch_prefill_simt<float>(q, k, v, g, beta, state_in, cu_seqlens, n_seqs, total_T, Hqk,
                                       Hv, dk, dv, scale, C, o, state_out, st);
+  if (dtype == GDN_F16)
+    return launch_prefill_simt<__half>(q, k, v, g, beta, state_in, cu_seqlens, n_seqs, total_T, Hqk,
+                                       Hv, dk, dv, scale, C, o, state_out, st);
   return launch_prefill_simt<__nv_bfloat16>(q, k, v, g, beta, state_in, cu_seqlens, n_seqs, total_T,
                                             Hqk, Hv, dk, dv, scale, C, o, state_out, st);
 }
@@ -439,6 +450,8 @@ gdn_status gdn_decode(const void* q, const void* k, const void* v, const float* 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dtype == GDN_F32)
     return dispatch_decode<float, float>(q, k, v, g, beta, state, B, Hqk, Hv, dk, dv, scale, o, st);
+  if (dtype == GDN_F16)
+    return dispatch_decode<__half, float>(q, k, v, g, beta, state, B, Hqk, Hv, dk, dv, scale, o, st);
   return dispatch_decode<__nv_bfloat16, float>(q, k, v, g, beta, state, B, Hqk, Hv, dk, dv, scale, o, st);
 }
 
@@ -455,6 +468,8 @@ gdn_status gdn_decode_bf16_state(const void* q, const void* k, const void* v, co
   auto* s16 = static_cast<__nv_bfloat16*>(state);
   if (dtype == GDN_F32)
     return dispatch_decode<float, __nv_bfloat16>(q, k, v, g, beta, s16, B, Hqk, Hv, dk, dv, scale, o, st);
+  if (dtype == GDN_F16)
+    return dispatch_decode<__half, __nv_bfloat16>(q, k, v, g, beta, s16, B, Hqk, Hv, dk, dv, scale, o, st);
   return dispatch_decode<__nv_bfloat16, __nv_bfloat16>(q, k, v, g, beta, s16, B, Hqk, Hv, dk, dv, scale, o, st);
 }
 
@@ -474,13 +489,29 @@ gdn_status gdn_device_error(void* stream) {
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "gdn_device_error: %s", cudaGetErrorString(e));
   if (word) {
+    unsigned int line = 0;
+    e = cudaMemcpyFromSymbolAsync(&line, gdn::g_error_line, sizeof line, 0, cudaMemcpyDeviceToHost, st);
     const unsigned int zero = 0;
-    e = cudaMemcpyToSymbolAsync(gdn::g_error_word, &zero, sizeof zero, 0, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess)
+      e = cudaMemcpyToSymbolAsync(gdn::g_error_word, &zero, sizeof zero, 0, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess)
+      e = cudaMemcpyToSymbolAsync(gdn::g_error_line, &zero, sizeof zero, 0, cudaMemcpyHostToDevice, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "gdn_device_error: %s", cudaGetErrorString(e));
+    if (word & gdn::kErrCheck)
+      return fail(GDN_ERR_DEVICE_CHECK, "an index check of the GDN_DEBUG build failed (source line %u, error word 0x%x)",
+                  line, word);
     return fail(GDN_ERR_DEVICE_TIMEOUT, "a bounded device wait ran out (error word 0x%x)", word);
   }
   return ok();
+}
+
+int gdn_debug_checks(void) {
+#ifdef GDN_DEBUG
+  return 1;
+#else
+  return 0;
+#endif
 }
 
 }  // extern "C"

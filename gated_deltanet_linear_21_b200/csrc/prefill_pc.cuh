@@ -1,6 +1,8 @@
 // Chunked Gated DeltaNet prefill on the sm_100a tensor cores, as one
-// persistent kernel with two kinds of CTA (bf16 inputs, d_k = d_v = 128,
-// chunk C = 64, fp32 state).
+// persistent kernel with two kinds of CTA (bf16 or f16 inputs, d_k = d_v =
+// 128, chunk C = 64, fp32 state). T is the 16-bit input type; every
+// tensor-core operand the kernel forms is rounded to T as well, so that no
+// product mixes the two formats, and accumulation is fp32 throughout.
 //
 // Algorithm: the WY (UT-transform) form of the gated delta rule. For a chunk
 // of L <= 64 tokens entering with state S, with G_r = sum_{s<=r} g_s,
@@ -98,8 +100,8 @@ constexpr int kMaxRounds = 1024;
 constexpr int kMaxPositions = 74;    // chains per round at most
 
 // ---- package: what a chain CTA needs from the preparation of one chunk ----
-constexpr uint32_t kPkgA1 = 0;        // A1 bf16 [128][128]: two K-major 128B-swizzled atoms, 16 KB apart
-constexpr uint32_t kPkgA2 = 32768;    // A2 bf16 [128][64]:  one K-major 128B-swizzled atom
+constexpr uint32_t kPkgA1 = 0;        // A1 T [128][128]: two K-major 128B-swizzled atoms, 16 KB apart
+constexpr uint32_t kPkgA2 = 32768;    // A2 T [128][64]:  one K-major 128B-swizzled atom
 constexpr uint32_t kPkgUs = 49152;    // us_r = exp(G_L - G_r) rk_r, fp32 [64]
 constexpr uint32_t kPkgGL = 49408;    // gamma_L fp32, tokens int
 constexpr uint32_t kPkgCopy = 49424;  // bytes copied per package (multiple of 16)
@@ -190,9 +192,8 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
                "r"(v.w)
                : "memory");
 }
-__device__ __forceinline__ void st_shared_b16(uint32_t addr, __nv_bfloat16 v) {
-  asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(*reinterpret_cast<unsigned short*>(&v))
-               : "memory");
+__device__ __forceinline__ void st_shared_u16(uint32_t addr, unsigned short v) {
+  asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
 }
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   uint4 v;
@@ -213,7 +214,7 @@ struct Params {
   const float* beta;
   const float* state_in;
   const int32_t* cu_seqlens;
-  __nv_bfloat16* o;
+  void* o;              // T [total_T][Hv][128]
   float* state_out;
   uint8_t* ws;          // workspace (counter and flags zeroed before the launch)
   int n_seqs, Hqk, Hv, total_T;
@@ -221,7 +222,7 @@ struct Params {
   int n_chain_ctas;     // CTAs [0, n_chain_ctas) run state chains, the rest prepare
 };
 
-template <int DVP>
+template <int DVP, typename T>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                   const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap omap,
@@ -229,6 +230,8 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
   using L = Smem<DVP>;
   using namespace sm100;
   static_assert(DVP == 32 || DVP == 64 || DVP == 128, "slice width");
+  constexpr uint32_t kFmt = Op16<T>::kFmt;   // every MMA operand is T: raw tiles and formed operands alike
+  T* const out = static_cast<T*>(p.o);
   constexpr int kSlices = kD / DVP;
   constexpr int kHalf = DVP / 2;
   constexpr uint32_t kR = L::kR, kRB = L::kRB;
@@ -243,7 +246,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
   uint64_t* bar_mma = bar_full + 4;
   uint64_t* bar_pub = bar_full + 5;                                  // [2] prep: publisher -> hand-over
   uint64_t* bar_u = bar_full + 5;      // chain: U_s staged (the 4 U warps)
-  uint64_t* bar_s = bar_full + 7;      // chain: the bf16 state copy is written
+  uint64_t* bar_s = bar_full + 7;      // chain: the 16-bit state copy is written
   uint32_t* misc = reinterpret_cast<uint32_t*>(sm + L::kMisc);     // [0] tmem, [2..5] scan
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -283,7 +286,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       uint32_t count = 1;
       if (is_chain && (i == 2 || i == 3)) count = 9;   // free: the 8 compute warps + the releasing warp
       if (is_chain && i == 5) count = 4;               // U_s staged: the 4 U warps
-      if (is_chain && i == 7) count = 8;               // bf16 state written: the 8 compute warps
+      if (is_chain && i == 7) count = 8;               // state copy written: the 8 compute warps
       mbar_init(&bar_full[i], count);
     }
     fence_mbar_init();
@@ -357,9 +360,15 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         const int hq = h / (Hv / Hqk);
         const int nch = (t_end - t_begin + kC - 1) / kC;
         const int maxc = round_maxc(j, q);
+        if (!GDN_CHECK(j < n_chains && h < Hv && hq < Hqk && i0 + DVP <= kD && q < chains_per_round &&
+                       0 <= t_begin && t_begin <= t_end && t_end <= p.total_T)) {
+          abort = true;
+          break;
+        }
         for (int c = 0; c < nch; ++c, ++gc) {
           const int b = (int)(gc & 1);
           const int s = base + c, slot = s % kRing;
+          if (!GDN_CHECK(s >= 0 && t_begin + c * kC < t_end)) { abort = true; break; }
           bool ok = true;
           if (lane == 0) ok = wait_flag_geq(&rdy[slot], (uint32_t)(s / kRing + 1));
           if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) { abort = true; break; }
@@ -390,6 +399,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         decode_sc(sc, j, h, i0, t_begin, t_end);
         const int nch = (t_end - t_begin + kC - 1) / kC;
         const int maxc = round_maxc(j, q);
+        if (!GDN_CHECK(q < chains_per_round && base >= 0 && maxc >= nch)) { abort = true; break; }
         for (int c = 0; c < nch; ++c, ++gc) {
           if (!mbar_wait(&bar_full[gc & 1], (uint32_t)(gc >> 1) & 1u)) { abort = true; break; }
           __syncwarp();
@@ -404,8 +414,8 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         base += maxc;
       }
     } else if (warp == kMmaWarp || warp < 8) {
-      constexpr uint32_t kIdY = idesc_bf16(128, DVP, false, true);
-      constexpr uint32_t kIdDS = idesc_bf16(128, DVP, true, true);
+      constexpr uint32_t kIdY = idesc_f16kind(128, DVP, false, true, kFmt);
+      constexpr uint32_t kIdDS = idesc_f16kind(128, DVP, true, true, kFmt);
       const uint32_t sSb = sbase + L::kSb;
       const uint32_t sUsb = sbase + L::kUsb;
       if (warp == kMmaWarp) {
@@ -417,7 +427,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           const uint32_t in = sbase + L::kIn + b * L::kInBytes;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_warp(tmem + ycol, desc_kmajor(in + kPkgA2, kk, 0), desc_mnmajor(in + L::kInV, kk, kRB, 64 * kRB),
+            mma_f16_warp(tmem + ycol, desc_kmajor(in + kPkgA2, kk, 0), desc_mnmajor(in + L::kInV, kk, kRB, 64 * kRB),
                           kIdY, kk > 0);
         };
         long gc = 0;
@@ -440,7 +450,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             if (c > 0 || p.state_in != nullptr) {   // (a first chunk from a zero state has no A1 S^T;
 #pragma unroll                                        //  its package carries no A1)
               for (int kk = 0; kk < 8; ++kk)
-                mma_bf16_warp(tmem + ycol, desc_kmajor(in + kPkgA1, kk, 16384), desc_mnmajor(sSb, kk, kRB, 128 * kRB),
+                mma_f16_warp(tmem + ycol, desc_kmajor(in + kPkgA1, kk, 16384), desc_mnmajor(sSb, kk, kRB, 128 * kRB),
                               kIdY, 1u);
             }
             mma_commit_warp(bar_mma);
@@ -450,7 +460,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              mma_bf16_warp(tmem + kColDS, desc_mnmajor(in + L::kInK, kk, 128, 8192),
+              mma_f16_warp(tmem + kColDS, desc_mnmajor(in + L::kInK, kk, 128, 8192),
                             desc_mnmajor(sUsb, kk, kRB, 64 * kRB), kIdDS, kk > 0);
             mma_commit_warp(bar_mma);
             // the other Y buffer was last read in chunk gc - 1, whose epilogues all ended
@@ -480,13 +490,18 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           const int nch = (t_end - t_begin + kC - 1) / kC;
 
           const size_t s_off = ((size_t)n * Hv + h) * kD * kD + (size_t)(i0 + ch * kHalf) * kD + r128;
+          if (!GDN_CHECK(n < p.n_seqs && h < Hv && i0 + DVP <= kD &&
+                         s_off + (size_t)(kHalf - 1) * kD < (size_t)p.n_seqs * Hv * kD * kD)) {
+            abort = true;
+            break;
+          }
           float Sreg[kHalf];
 #pragma unroll
           for (int q2 = 0; q2 < kHalf; ++q2) Sreg[q2] = p.state_in ? p.state_in[s_off + (size_t)q2 * kD] : 0.f;
           auto store_state = [&]() {
 #pragma unroll
             for (int c8 = 0; c8 < kHalf / 8; ++c8)
-              st_shared_v4(sSb + L::tile_off(r128, ch * kHalf + 8 * c8, 128), pack8_bf16(Sreg + 8 * c8));
+              st_shared_v4(sSb + L::tile_off(r128, ch * kHalf + 8 * c8, 128), pack8<T>(Sreg + 8 * c8));
           };
           if (nch > 0) {
             store_state();
@@ -501,29 +516,30 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             const bool full_ok = mbar_wait(&bar_full[b], (uint32_t)(gc >> 1) & 1u);
             const int len = min(kC, t_end - (t_begin + c * kC));
             const bool o_tma = len == kC;
+            if (!GDN_CHECK(len > 0 && t_begin + c * kC + len <= p.total_T)) { abort = true; break; }
             if (!wait_mma(full_ok)) { abort = true; break; }   // Y
             {
               const float us = qd < 2 ? reinterpret_cast<const float*>(in_g + kPkgUs)[r128] : 0.f;
-              __nv_bfloat16* orow = p.o + ((size_t)(t_begin + c * kC + (r128 & 63)) * Hv + h) * kD + i0 + ch * kHalf;
+              T* orow = out + ((size_t)(t_begin + c * kC + (r128 & 63)) * Hv + h) * kD + i0 + ch * kHalf;
 #pragma unroll
               for (int pp = 0; pp < kHalf / kPart; ++pp) {
                 float yv[kPart];
                 tmem_ld<kPart>(tmem + tlane + kColY + 128u * (uint32_t)b + ch * kHalf + pp * kPart, yv);
-                if (qd < 2) {   // U_s = diag(us) U -> shared memory (bf16) for dS
+                if (qd < 2) {   // U_s = diag(us) U -> shared memory (T) for dS
 #pragma unroll
                   for (int q2 = 0; q2 < kPart; ++q2) yv[q2] *= us;
 #pragma unroll
                   for (int c8 = 0; c8 < kPart / 8; ++c8)
-                    st_shared_v4(sUsb + L::tile_off(r128, ch * kHalf + pp * kPart + 8 * c8, 64), pack8_bf16(yv + 8 * c8));
+                    st_shared_v4(sUsb + L::tile_off(r128, ch * kHalf + pp * kPart + 8 * c8, 64), pack8<T>(yv + 8 * c8));
                 } else if (o_tma) {   // O staged in the consumed v tile for the TMA store
 #pragma unroll
                   for (int c8 = 0; c8 < kPart / 8; ++c8)
                     st_shared_v4(in + L::kInV + L::tile_off(r128 - 64, ch * kHalf + pp * kPart + 8 * c8, 64),
-                                 pack8_bf16(yv + 8 * c8));
+                                 pack8<T>(yv + 8 * c8));
                 } else if (r128 - 64 < len) {   // a sequence's last, partial chunk: row by row
 #pragma unroll
                   for (int c8 = 0; c8 < kPart / 8; ++c8)
-                    *reinterpret_cast<uint4*>(orow + pp * kPart + 8 * c8) = pack8_bf16(yv + 8 * c8);
+                    *reinterpret_cast<uint4*>(orow + pp * kPart + 8 * c8) = pack8<T>(yv + 8 * c8);
                 }
               }
             }
@@ -630,6 +646,9 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             q = local % cpr;
             j = j0 + q;
             s = rbase[r] + c;
+            if (!GDN_CHECK(r >= 0 && r < n_rounds && cpr > 0 && local >= 0 && q < chains_per_round &&
+                           j < n_chains && s >= 0))
+              break;
             if (c < n_chunks_of(j)) { v = 1; break; }
           }
         }
@@ -648,6 +667,10 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           len = min(kC, te - c0);
           // the raw k, q tiles first: their latency covers the gates and the slot wait
           const int hq = h / (Hv / Hqk);
+          if (!GDN_CHECK(0 <= c0 && len > 0 && c0 + len <= p.total_T && h < Hv && hq < Hqk)) {
+            len = 0;   // (no gate is read; the tile loads below stay inside their tensor maps)
+            v = 0;
+          }
           uint8_t* kq = sm + L::kKQP + b * 32768;
           mbar_expect_tx_warp(&bar_full[b], 4 * 8192);
           tma_load_3d_warp(kq, &kmap, &bar_full[b], 0, hq, c0);
@@ -665,7 +688,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           if (lane == 0 && s >= kRing) ok = wait_flag_geq(&consumed[q * kRing + s % kRing], (uint32_t)(kSlices * (s / kRing)));
           ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         }
-        const bool go = v && ok;
+        const bool go = v && ok && len > 0;
         if (lane == 0) {
           qe[0] = go ? 1u : 0u;
           qe[1] = (uint32_t)s;
@@ -693,6 +716,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         if (!mbar_wait(&bar_full[b], par)) break;   // handed over (or the end marker)
         const uint32_t* qe = reinterpret_cast<const uint32_t*>(sm + L::kQueue + b * L::kQueueBytes);
         if (qe[0] == 0) break;
+        if (!GDN_CHECK(qe[2] < (uint32_t)chains_per_round)) break;
         if (!mbar_wait(&bar_free[b], par)) break;
         if (lane == 0) st_release_gpu(&ready[qe[2] * kRing + qe[1] % kRing], qe[1] / kRing + 1);
         __syncwarp();
@@ -700,8 +724,8 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       }
     } else if (warp < 8) {
       // ---- compute warps (warp 10 has no job in a prep CTA) ----
-      constexpr uint32_t kIdG = idesc_bf16(128, 64, false, false);
-      constexpr uint32_t kId64 = idesc_bf16(64, 64, false, true);
+      constexpr uint32_t kIdG = idesc_f16kind(128, 64, false, false, kFmt);
+      constexpr uint32_t kId64 = idesc_f16kind(64, 64, false, true, kFmt);
       float* vG = reinterpret_cast<float*>(sm + L::kVec);   // per-warp partial scan of g
       float* vB = vG + 64;
       float* vRk = vB + 64;
@@ -738,6 +762,12 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         }
         if (qe[0] == 0) break;
         const int len = (int)qe[3];
+#ifdef GDN_DEBUG
+        if (!cbar_and(GDN_CHECK(qe[2] < (uint32_t)chains_per_round && len > 0 && len <= kC))) {
+          abort = true;
+          break;
+        }
+#endif
         // a chain's first chunk from a zero state never multiplies A1 (S = 0): skip -W, P W
         const bool need_a1 = qe[4] != 0 || p.state_in != nullptr;
         uint8_t* pkg = pkgs + ((size_t)qe[2] * kRing + qe[1] % kRing) * kPkgStride;
@@ -747,7 +777,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         if (warp == 0) {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_bf16_warp(tmem + kColG, desc_kmajor(sKQ, kk, 16384), desc_kmajor(sKQ, kk, 16384), kIdG, kk > 0);
+            mma_f16_warp(tmem + kColG, desc_kmajor(sKQ, kk, 16384), desc_kmajor(sKQ, kk, 16384), kIdG, kk > 0);
           mma_commit_warp(bar_mma);
         } else if (tid == kOutThread) {
           finish_out();   // (before this item's vectors reuse the staging)
@@ -770,13 +800,12 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           float ss0 = 0.f, ss1 = 0.f;
 #pragma unroll
           for (int c8 = 0; c8 < 16; ++c8) {
-            const uint4 raw = ld_shared_v4(sKQ + sw128_off(row, 8 * c8, 16384));
-            const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+            float f[8];
+            unpack8<T>(ld_shared_v4(sKQ + sw128_off(row, 8 * c8, 16384)), f);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float2 f = __bfloat1622float2(p2[e]);
-              if (e & 1) ss1 = fmaf(f.x, f.x, fmaf(f.y, f.y, ss1));
-              else ss0 = fmaf(f.x, f.x, fmaf(f.y, f.y, ss0));
+              if (e & 1) ss1 = fmaf(f[2 * e], f[2 * e], fmaf(f[2 * e + 1], f[2 * e + 1], ss1));
+              else ss0 = fmaf(f[2 * e], f[2 * e], fmaf(f[2 * e + 1], f[2 * e + 1], ss0));
             }
           }
           const float ss = ss0 + ss1;
@@ -808,7 +837,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         }
         if (!wait_mma()) { abort = true; break; }   // (its barrier also publishes the vectors)
 
-        // ---- A (diagonal blocks fp32, off-diagonal blocks bf16) and P ----
+        // ---- A (diagonal blocks fp32, off-diagonal blocks T) and P ----
         {
           float gram[32];
           tmem_ld32(tmem + tlane + kColG + 32 * ch, gram);
@@ -854,7 +883,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             for (int q2 = 0; q2 < 32; ++q2) x[q2] = (32 * ch + q2 < 16 * blk) ? x[q2] : 0.f;
 #pragma unroll
             for (int c8 = 0; c8 < 4; ++c8)
-              st_shared_v4(sbase + L::kAo + sw128_off(rr, 32 * ch + 8 * c8, 0), pack8_bf16(x + 8 * c8));
+              st_shared_v4(sbase + L::kAo + sw128_off(rr, 32 * ch + 8 * c8, 0), pack8<T>(x + 8 * c8));
           } else {
             const float fr = vRq[rr] * (fast ? expf(Gr - gm) : 1.f);
             if (fast) {
@@ -872,7 +901,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             }
 #pragma unroll
             for (int c8 = 0; c8 < 4; ++c8)
-              st_shared_v4(sbase + L::kPm + sw128_off(rr, 32 * ch + 8 * c8, 0), pack8_bf16(x + 8 * c8));
+              st_shared_v4(sbase + L::kPm + sw128_off(rr, 32 * ch + 8 * c8, 0), pack8<T>(x + 8 * c8));
           }
         }
         cbar();
@@ -895,7 +924,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           }
 #pragma unroll
           for (int i = 0; i < 16; ++i)
-            st_shared_b16(sbase + L::kDm + sw128_off(16 * blk + i, 16 * blk + jj, 0), __float2bfloat16_rn(xs[i]));
+            st_shared_u16(sbase + L::kDm + sw128_off(16 * blk + i, 16 * blk + jj, 0), Op16<T>::one(xs[i]));
         } else {
           for (int e = tid - 64; e < 64 * 6; e += kCompute - 64) {
             const int row = e / 6, idx = e - row * 6, blk = row >> 4;
@@ -909,7 +938,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         if (warp == 0) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_warp(tmem + kColN, desc_kmajor(sbase + L::kDm, kk, 0), desc_mnmajor(sbase + L::kAo, kk, 128, 8192),
+            mma_f16_warp(tmem + kColN, desc_kmajor(sbase + L::kDm, kk, 0), desc_mnmajor(sbase + L::kAo, kk, 128, 8192),
                           kId64, kk > 0);
           mma_commit_warp(bar_mma);
         }
@@ -920,7 +949,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           if (lo16) {
 #pragma unroll
             for (int c8 = 0; c8 < 4; ++c8)
-              st_shared_v4(sbase + L::kNm + sw128_off(r64, 32 * ch + 8 * c8, 0), pack8_bf16(v + 8 * c8));
+              st_shared_v4(sbase + L::kNm + sw128_off(r64, 32 * ch + 8 * c8, 0), pack8<T>(v + 8 * c8));
           }
         }
         publish();
@@ -929,11 +958,11 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         if (warp == 0) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_warp(tmem + kColS2, desc_kmajor(sbase + L::kNm, kk, 0),
+            mma_f16_warp(tmem + kColS2, desc_kmajor(sbase + L::kNm, kk, 0),
                           desc_mnmajor(sbase + L::kDm, kk, 128, 8192), kId64, kk > 0);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_warp(tmem + (16u << 16) + kColS2, desc_kmajor(sbase + L::kNm, kk, 0),
+            mma_f16_warp(tmem + (16u << 16) + kColS2, desc_kmajor(sbase + L::kNm, kk, 0),
                           desc_mnmajor(sbase + L::kNm, kk, 128, 8192), kId64, kk > 0);
           mma_commit_warp(bar_mma);
         }
@@ -945,20 +974,16 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           if (lo16) {
 #pragma unroll
             for (int c8 = 0; c8 < 4; ++c8) {
-              const uint4 dv = ld_shared_v4(sbase + L::kDm + sw128_off(r64, 32 * ch + 8 * c8, 0));
-              const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
+              float df[8];
+              unpack8<T>(ld_shared_v4(sbase + L::kDm + sw128_off(r64, 32 * ch + 8 * c8, 0)), df);
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float2 df = __bfloat1622float2(d2[e]);
-                E[8 * c8 + 2 * e] = df.x - v[8 * c8 + 2 * e];
-                E[8 * c8 + 2 * e + 1] = df.y - v[8 * c8 + 2 * e + 1];
-              }
-              st_shared_v4(sbase + L::kEm + sw128_off(r64, 32 * ch + 8 * c8, 0), pack8_bf16(E + 8 * c8));
+              for (int e = 0; e < 8; ++e) E[8 * c8 + e] = df[e] - v[8 * c8 + e];
+              st_shared_v4(sbase + L::kEm + sw128_off(r64, 32 * ch + 8 * c8, 0), pack8<T>(E + 8 * c8));
             }
           } else {
 #pragma unroll
             for (int c8 = 0; c8 < 4; ++c8)
-              st_shared_v4(sbase + L::kN2 + sw128_off(r64, 32 * ch + 8 * c8, 0), pack8_bf16(v + 8 * c8));
+              st_shared_v4(sbase + L::kN2 + sw128_off(r64, 32 * ch + 8 * c8, 0), pack8<T>(v + 8 * c8));
           }
         }
         publish();
@@ -967,7 +992,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         if (warp == 0) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_warp(tmem + kColZ, desc_kmajor(sbase + L::kN2, kk, 0), desc_mnmajor(sbase + L::kEm, kk, 128, 8192),
+            mma_f16_warp(tmem + kColZ, desc_kmajor(sbase + L::kN2, kk, 0), desc_mnmajor(sbase + L::kEm, kk, 128, 8192),
                           kId64, kk > 0);
           mma_commit_warp(bar_mma);
         }
@@ -987,8 +1012,8 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
                 tw[e] = t * vCw[sidx];
               }
               const uint32_t off = sw128_off(r64, 32 * ch + 8 * c8, 0);
-              st_shared_v4(sbase + L::kTu + off, pack8_bf16(tu));
-              st_shared_v4(sbase + L::kTw + off, pack8_bf16(tw));
+              st_shared_v4(sbase + L::kTu + off, pack8<T>(tu));
+              st_shared_v4(sbase + L::kTw + off, pack8<T>(tw));
             }
           }
         }
@@ -1001,11 +1026,11 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           if (warp == 0) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              mma_bf16_warp(tmem + kColW, desc_kmajor(sbase + L::kTw, kk, 0), desc_mnmajor(sKQ, kk, 128, 16384), kId64,
+              mma_f16_warp(tmem + kColW, desc_kmajor(sbase + L::kTw, kk, 0), desc_mnmajor(sKQ, kk, 128, 16384), kId64,
                             kk > 0);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              mma_bf16_warp(tmem + (16u << 16) + kColW, desc_kmajor(sbase + L::kTw, kk, 0),
+              mma_f16_warp(tmem + (16u << 16) + kColW, desc_kmajor(sbase + L::kTw, kk, 0),
                             desc_mnmajor(sKQ + 16384, kk, 128, 16384), kId64, kk > 0);
             mma_commit_warp(bar_mma);
           }
@@ -1015,7 +1040,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             tmem_ld32(tmem + tlane + kColW + 32 * ch, w);
 #pragma unroll
             for (int c8 = 0; c8 < 4; ++c8)
-              st_shared_v4(sbase + L::kWm + sw128_off(r64, dhalf + 8 * c8, 8192), pack8_bf16(w + 8 * c8));
+              st_shared_v4(sbase + L::kWm + sw128_off(r64, dhalf + 8 * c8, 8192), pack8<T>(w + 8 * c8));
           }
           publish();
         }
@@ -1025,16 +1050,16 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           if (need_a1) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              mma_bf16_warp(tmem + kColPW, desc_kmajor(sbase + L::kPm, kk, 0),
+              mma_f16_warp(tmem + kColPW, desc_kmajor(sbase + L::kPm, kk, 0),
                             desc_mnmajor(sbase + L::kWm, kk, 128, 8192), kId64, kk > 0);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              mma_bf16_warp(tmem + (16u << 16) + kColPW, desc_kmajor(sbase + L::kPm, kk, 0),
+              mma_f16_warp(tmem + (16u << 16) + kColPW, desc_kmajor(sbase + L::kPm, kk, 0),
                             desc_mnmajor(sbase + L::kWm + 8192, kk, 128, 8192), kId64, kk > 0);
           }
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_warp(tmem + kColPT, desc_kmajor(sbase + L::kPm, kk, 0), desc_mnmajor(sbase + L::kTu, kk, 128, 8192),
+            mma_f16_warp(tmem + kColPT, desc_kmajor(sbase + L::kPm, kk, 0), desc_mnmajor(sbase + L::kTu, kk, 128, 8192),
                           kId64, kk > 0);
           mma_commit_warp(bar_mma);
         }
@@ -1047,16 +1072,11 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
 #pragma unroll
             for (int c8 = 0; c8 < 4; ++c8) {
               const int d = dhalf + 8 * c8;
-              const uint4 qv = ld_shared_v4(sKQ + sw128_off(64 + r64, d, 16384));
-              const __nv_bfloat162* q2v = reinterpret_cast<const __nv_bfloat162*>(&qv);
-              float a[8];
+              float qf[8], a[8];
+              unpack8<T>(ld_shared_v4(sKQ + sw128_off(64 + r64, d, 16384)), qf);
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float2 qf = __bfloat1622float2(q2v[e]);
-                a[2 * e] = fmaf(rho, qf.x, pw[8 * c8 + 2 * e]);
-                a[2 * e + 1] = fmaf(rho, qf.y, pw[8 * c8 + 2 * e + 1]);
-              }
-              st_shared_v4(sbase + L::kA1b + sw128_off(r64, d, 8192), pack8_bf16(a));
+              for (int e = 0; e < 8; ++e) a[e] = fmaf(rho, qf[e], pw[8 * c8 + e]);
+              st_shared_v4(sbase + L::kA1b + sw128_off(r64, d, 8192), pack8<T>(a));
             }
           }
           float pt[32];
@@ -1064,7 +1084,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           if (lo16) {
 #pragma unroll
             for (int c8 = 0; c8 < 4; ++c8)
-              st_shared_v4(sbase + L::kA2b + sw128_off(r64, 32 * ch + 8 * c8, 0), pack8_bf16(pt + 8 * c8));
+              st_shared_v4(sbase + L::kA2b + sw128_off(r64, 32 * ch + 8 * c8, 0), pack8<T>(pt + 8 * c8));
           }
         }
         // ---- the package images are complete: copy them out in bulk; the copies are

@@ -7,9 +7,9 @@
 // byte offset >> 4 in [32,46), descriptor version 1 at bit 46, swizzle mode
 // in [61,64) (2 = 128-byte, 4 = 64-byte, 6 = 32-byte). Canonical layouts
 // (bytes; a "row" is one 16/32/64/128-byte swizzle row):
-//   K-major, 128B swizzle : rows of 64 bf16 along K, 8-row groups 1024 B apart
+//   K-major, 128B swizzle : rows of 64 16-bit values along K, 8-row groups 1024 B apart
 //                           (stride offset), 16-byte chunk index XOR (row & 7).
-//   MN-major, S-byte swizzle: rows of S/2 bf16 along M/N, one row per K index,
+//   MN-major, S-byte swizzle: rows of S/2 16-bit values along M/N, one row per K index,
 //                           8 K-rows per group (stride offset = 8 * S), further
 //                           blocks of S/2 M/N elements at the leading offset.
 // Every swizzled tile starts on a 1024-byte boundary.
@@ -221,8 +221,9 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem], bf16 inputs, fp32 accumulate; one K=16 step.
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+// D[tmem] (+)= A[smem] * B[smem], kind::f16: 16-bit inputs (both f16 or both bf16,
+// as the instruction descriptor says), fp32 accumulate; one K=16 step.
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                          uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
@@ -237,7 +238,7 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
 // from a single divergent thread costs tens to hundreds of cycles per
 // instruction. The elected lane is the lowest active one, so a commit made
 // the same way tracks the MMAs issued by the same lane.
-__device__ __forceinline__ void mma_bf16_warp(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+__device__ __forceinline__ void mma_f16_warp(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                               uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred e, p;\n\t"
@@ -292,16 +293,20 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
                : "memory");
 }
 
-// Instruction descriptor, kind::f16 with bf16 A/B and fp32 D.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
+// Instruction descriptor, kind::f16 with fp32 D and A, B both of the 16-bit
+// type whose format code is `ab_fmt` (0 = f16, 1 = bf16; one MMA never mixes
+// the two).
+__host__ __device__ constexpr uint32_t idesc_f16kind(int M, int N, bool a_mn_major, bool b_mn_major,
+                                                     uint32_t ab_fmt) {
   return (1u << 4)                                   // D format f32
-         | (1u << 7)                                 // A format bf16
-         | (1u << 10)                                // B format bf16
+         | (ab_fmt << 7)                             // A format
+         | (ab_fmt << 10)                            // B format
          | (static_cast<uint32_t>(a_mn_major) << 15) //
          | (static_cast<uint32_t>(b_mn_major) << 16) //
          | (static_cast<uint32_t>(N >> 3) << 17)     //
          | (static_cast<uint32_t>(M >> 4) << 24);
 }
+
 
 enum : uint32_t { kSwizzle128 = 2, kSwizzle64 = 4, kSwizzle32 = 6 };
 
@@ -313,7 +318,7 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
          (static_cast<uint64_t>(swizzle) << 61);
 }
 
-// Descriptor for K-step `kk` (16 bf16) of a K-major 128B-swizzled operand whose
+// Descriptor for K-step `kk` (16 elements) of a K-major 128B-swizzled operand whose
 // 64-element atom columns are `acs` bytes apart.
 __device__ __forceinline__ uint64_t desc_kmajor(uint32_t base, int kk, uint32_t acs) {
   return smem_desc(base + (kk >> 2) * acs + (kk & 3) * 32, 16, 1024, kSwizzle128);
@@ -430,18 +435,48 @@ __device__ __forceinline__ void tmem_ld(uint32_t taddr, float* r) {
   }
 }
 
-// Pack 8 floats into 8 bf16 (round to nearest even) as one 16-byte chunk.
-__device__ __forceinline__ uint4 pack8_bf16(const float* x) {
-  uint4 out;
-  __nv_bfloat162 a = __floats2bfloat162_rn(x[0], x[1]);
-  __nv_bfloat162 b = __floats2bfloat162_rn(x[2], x[3]);
-  __nv_bfloat162 c = __floats2bfloat162_rn(x[4], x[5]);
-  __nv_bfloat162 d = __floats2bfloat162_rn(x[6], x[7]);
-  out.x = *reinterpret_cast<uint32_t*>(&a);
-  out.y = *reinterpret_cast<uint32_t*>(&b);
-  out.z = *reinterpret_cast<uint32_t*>(&c);
-  out.w = *reinterpret_cast<uint32_t*>(&d);
-  return out;
+// The 16-bit tensor-core operand types (kind::f16): format code, packing of 8
+// floats into one 16-byte chunk (round to nearest even) and unpacking.
+template <typename T> struct Op16;
+template <> struct Op16<__nv_bfloat16> {
+  static constexpr uint32_t kFmt = 1u;
+  static __device__ __forceinline__ uint32_t pack2(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+  static __device__ __forceinline__ float2 unpack2(uint32_t u) {
+    return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u));
+  }
+  static __device__ __forceinline__ unsigned short one(float x) {
+    __nv_bfloat16 h = __float2bfloat16_rn(x);
+    return *reinterpret_cast<unsigned short*>(&h);
+  }
+};
+template <> struct Op16<__half> {
+  static constexpr uint32_t kFmt = 0u;
+  static __device__ __forceinline__ uint32_t pack2(float a, float b) {
+    __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+  static __device__ __forceinline__ float2 unpack2(uint32_t u) {
+    return __half22float2(*reinterpret_cast<__half2*>(&u));
+  }
+  static __device__ __forceinline__ unsigned short one(float x) {
+    __half h = __float2half_rn(x);
+    return *reinterpret_cast<unsigned short*>(&h);
+  }
+};
+template <typename T>
+__device__ __forceinline__ uint4 pack8(const float* x) {
+  return make_uint4(Op16<T>::pack2(x[0], x[1]), Op16<T>::pack2(x[2], x[3]), Op16<T>::pack2(x[4], x[5]),
+                    Op16<T>::pack2(x[6], x[7]));
+}
+// The 8 values of a 16-byte chunk of T as floats.
+template <typename T>
+__device__ __forceinline__ void unpack8(uint4 v, float* x) {
+  const float2 a = Op16<T>::unpack2(v.x), b = Op16<T>::unpack2(v.y), c = Op16<T>::unpack2(v.z),
+               d = Op16<T>::unpack2(v.w);
+  x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y; x[4] = c.x; x[5] = c.y; x[6] = d.x; x[7] = d.y;
 }
 
 }  // namespace sm100

@@ -29,8 +29,12 @@
  *     The caller owns every buffer; the library never allocates, frees or
  *     synchronises (except gdn_device_error, which synchronises the stream).
  *   - dtype GDN_BF16: q, k, v, o are bf16 (o rounded to nearest even from
- *     fp32). GDN_F32: q, k, v, o are fp32. g and beta are fp32 in both
- *     cases, and so are the states, except in gdn_decode_bf16_state.
+ *     fp32). GDN_F16: q, k, v, o are IEEE f16 (o rounded to nearest even),
+ *     the pages' second numerical mode ("One level down: #004 the same
+ *     compiler on Apple's chips", section "f16"); values beyond the f16
+ *     range are the caller's concern. GDN_F32: q, k, v, o are fp32. g and
+ *     beta are fp32 in every case, and so are the states, except in
+ *     gdn_decode_bf16_state. Arithmetic is fp32 accumulation throughout.
  *   - Grouped heads: Hv must be a multiple of Hqk; value head h reads
  *     query/key head floor(h / (Hv / Hqk)) (contiguous groups).
  *   - g is the log-decay ln(alpha) (<= 0 in normal use); beta is used as given.
@@ -59,12 +63,14 @@ typedef enum gdn_status {
     GDN_ERR_INVALID_ARG = 1,    /* null pointer, bad size, misaligned pointer, bad cu_seqlens */
     GDN_ERR_UNSUPPORTED = 2,    /* valid but unsupported shape/dtype combination */
     GDN_ERR_CUDA = 3,           /* a CUDA call or launch failed */
-    GDN_ERR_DEVICE_TIMEOUT = 4  /* a bounded device-side wait ran out (gdn_device_error) */
+    GDN_ERR_DEVICE_TIMEOUT = 4, /* a bounded device-side wait ran out (gdn_device_error) */
+    GDN_ERR_DEVICE_CHECK = 5    /* an index check of the GDN_DEBUG build failed (gdn_device_error) */
 } gdn_status;
 
 typedef enum gdn_dtype {
-    GDN_BF16 = 0,
-    GDN_F32 = 1
+    GDN_BF16 = 0,   /* bfloat16 */
+    GDN_F32 = 1,    /* IEEE binary32 */
+    GDN_F16 = 2     /* IEEE binary16 */
 } gdn_dtype;
 
 /*
@@ -87,7 +93,7 @@ int gdn_version(void);
 
 /*
  * Bytes of device workspace gdn_prefill needs for this problem: 0 unless the
- * tensor-core kernel runs it (GDN_BF16, dk = dv = 128). The tensor-core
+ * tensor-core kernel runs it (GDN_BF16 or GDN_F16, dk = dv = 128). The tensor-core
  * kernel splits its CTAs into ones that prepare, per (value head, chunk), the
  * state-independent operands of the chunk and ones that carry the state from
  * chunk to chunk; the workspace holds the ring of prepared packages between
@@ -111,8 +117,8 @@ size_t gdn_prefill_workspace_bytes(int n_seqs, int Hv, int dk, int dv, gdn_dtype
  * Host only: touches no device memory and launches nothing (with sm_count > 0
  * it needs no GPU at all).
  * Returns GDN_ERR_UNSUPPORTED where the tensor-core kernel does not run
- * (dtype other than GDN_BF16, or dk, dv other than 128: those shapes run on
- * the fp32 SIMT kernel) and GDN_ERR_INVALID_ARG for a null output, an invalid
+ * (GDN_F32, or dk, dv other than 128: those shapes run on the fp32 SIMT
+ * kernel) and GDN_ERR_INVALID_ARG for a null output, an invalid
  * request, n_seqs or Hv <= 0, total_T < 0, or fewer than 16 multiprocessors.
  */
 gdn_status gdn_prefill_plan(int n_seqs, int64_t total_T, int Hv, int dk, int dv, gdn_dtype dtype, int sm_count,
@@ -135,9 +141,11 @@ gdn_status gdn_prefill_plan(int n_seqs, int64_t total_T, int Hv, int dk, int dv,
  *              dk = dv = 128, else 16). The result does not depend on it
  *              beyond rounding.
  *
- * Supported: GDN_BF16 with dk = dv = 128 and chunk 64 (tensor-core kernel);
- * GDN_F32 (and GDN_BF16 with other sizes) with dk, dv in {16, 32, 64, 128}
- * and chunk in {16, 32, 64} (fp32 SIMT kernel). total_T < 2^31. The
+ * Supported: GDN_BF16 or GDN_F16 with dk = dv = 128 and chunk 64
+ * (tensor-core kernel: every tensor-core operand in the input's 16-bit
+ * format, fp32 accumulation and state); GDN_F32 (and the 16-bit types with
+ * other sizes or chunks) with dk, dv in {16, 32, 64, 128} and chunk in
+ * {16, 32, 64} (fp32 SIMT kernel). total_T < 2^31. The
  * tensor-core kernel runs the sequence-heads in at most 1024 rounds of up to
  * 74 at a time; larger problems return GDN_ERR_UNSUPPORTED (split them
  * across calls). It is one cooperative launch with one CTA on every SM of the
@@ -223,7 +231,7 @@ gdn_status gdn_prefill_noalloc(const void *q, const void *k, const void *v,
  *   state   [B, Hv, dv, dk]  fp32, updated in place
  *   o       [B, Hv, dv]      dtype (output)
  *
- * Supported: dk and dv in {16, 32, 64, 128}, either dtype.
+ * Supported: dk and dv in {16, 32, 64, 128}, any dtype.
  */
 gdn_status gdn_decode(const void *q, const void *k, const void *v,
                       const float *g, const float *beta, float *state,
@@ -264,11 +272,25 @@ const char *gdn_last_error(void);
 
 /*
  * Synchronise `stream` and read, then clear, the device error word of the
- * current device. Returns GDN_ERR_DEVICE_TIMEOUT if a bounded wait ran out
- * in any kernel since the last call, GDN_ERR_CUDA if synchronisation failed,
- * else GDN_OK. Meant for tests and debugging; not needed in normal use.
+ * current device. Returns GDN_ERR_DEVICE_CHECK if an index check of a
+ * GDN_DEBUG build failed (the message names the check's source line),
+ * GDN_ERR_DEVICE_TIMEOUT if a bounded wait ran out in any kernel since the
+ * last call, GDN_ERR_CUDA if synchronisation failed, else GDN_OK. Meant for
+ * tests and debugging; not needed in normal use.
  */
 gdn_status gdn_device_error(void *stream);
+
+/*
+ * 1 if this library was built with GDN_DEBUG (libgdn_debug.so), else 0. The
+ * debug build checks, on the device, the ring positions and slots, sequence
+ * bounds, token and head coordinates and state offsets that the tensor-core
+ * prefill computes before it uses them; a failed check records
+ * GDN_ERR_DEVICE_CHECK in the device error word and stops that CTA's work
+ * (the waits of the others are bounded), instead of reading or writing out
+ * of bounds. It never traps. Diagnostic only: the checks cost time, and the
+ * pages have no counterpart. Same ABI as the normal build otherwise.
+ */
+int gdn_debug_checks(void);
 
 #ifdef __cplusplus
 }

@@ -127,6 +127,10 @@ def test_prefill_plan_for_the_benchmark_workloads():
     # long prompts x 32 heads: 32 chains of one 128-row slice, 116 preparing CTAs
     assert gdn.prefill_plan(1, 32768, 32, sm_count=148) == (128, 32, 1)
     assert gdn.prefill_plan(1, 81920, 32, sm_count=148) == (128, 32, 1)
+    # f16 inputs run the same kernel with the same plans and workspace
+    assert gdn.prefill_plan(1, 4096, 16, dtype=torch.float16, sm_count=148) == (32, 64, 1)
+    assert gdn.prefill_workspace_bytes(1, 16, 128, 128, torch.float16) == \
+        gdn.prefill_workspace_bytes(1, 16, 128, 128, torch.bfloat16) > 0
 
 
 @pytest.mark.parametrize("n_seqs,total_T,Hv", [(8, 37000, 32), (300, 45000, 8), (3, 500, 8), (64, 64 * 300, 16)])

@@ -118,6 +118,17 @@ def test_tensor_core_prefill_edges(kind, L):
     _compare(f"{kind} L={L} state", s, rs, 1e-2)
 
 
+@pytest.mark.parametrize("kind", ("strong_decay", "no_decay", "positive_g", "zero_qk", "mixed_chunks"))
+def test_tensor_core_prefill_edges_f16(kind):
+    """The f16 instantiation of the tensor-core kernel on the same edges (its
+    operands have a narrower exponent range than bf16: tiny decayed terms
+    flush to zero)."""
+    x = edge_inputs(kind, 197, dtype=torch.float16)
+    o, s, ro, rs = _run(x)
+    _compare(f"{kind} f16 o", o, ro, 2e-2)
+    _compare(f"{kind} f16 state", s, rs, 1e-2)
+
+
 @pytest.mark.parametrize("kind", KINDS)
 def test_simt_prefill_edges_fp32(kind):
     x = edge_inputs(kind, 197, d=64, dtype=torch.float32)

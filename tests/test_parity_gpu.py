@@ -96,14 +96,14 @@ def check_prefill(x, tol_o, tol_s, chunk=0, heads=None, alias=False, plan=None):
 
 # ------------------------------------------------------------------ decode ---
 
-@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16, torch.float32])
 @pytest.mark.parametrize("dk,dv", [(16, 16), (32, 64), (64, 128), (128, 128), (128, 32)])
 def test_decode_small(dtype, dk, dv):
     B, Hqk, Hv = 3, 2, 4
     state = workloads.decode_state(B, Hv, dk, std=0.05, dv=dv)
     ref_state = state.double().numpy().copy()
     sd = state.to(DEV)
-    tol = 2e-2 if dtype == torch.bfloat16 else 1e-5
+    tol = 2e-2 if dtype != torch.float32 else 1e-5
     for step in range(5):
         x = workloads.decode_step_inputs(step, B, Hqk, Hv, dk, dtype, dv=dv)
         o = torch.full((B, Hv, dv), float("nan"), dtype=dtype, device=DEV)
@@ -113,7 +113,7 @@ def test_decode_small(dtype, dk, dv):
         eo, mo = _max_err(o, ro)
         _gate("o", eo, mo, tol)
     es, ms = _max_err(sd, ref_state)
-    _gate("state", es, ms, 1e-2 if dtype == torch.bfloat16 else 1e-5)
+    _gate("state", es, ms, 1e-2 if dtype != torch.float32 else 1e-5)
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
@@ -178,6 +178,97 @@ def test_decode_bf16_state_workload_1000_steps_sampled_heads():
     _gate("state", es, ms, w.tol_state)
 
 
+def test_decode_workload_f16_1000_steps_sampled_heads():
+    """The decode workload (64 sequences x 32 value heads, 1000 steps) with f16
+    q, k, v and o and the fp32 state, on value heads 0, 13 and 31, at the
+    workload's tolerances and the 1/64 gate."""
+    w = workloads.workload("decode")
+    sel = (slice(None), DECODE_HEADS)
+    state = workloads.decode_state(w.batch, w.Hv, w.d, std=w.state_std)
+    ref = state.double().numpy().copy()
+    sd = state.to(DEV)
+    worst_o = 0.0
+    for step in range(w.steps):
+        x = workloads.decode_step_inputs(step, w.batch, w.Hqk, w.Hv, w.d, dtype=torch.float16)
+        o = gdn.decode(x["q"].to(DEV), x["k"].to(DEV), x["v"].to(DEV), x["g"].to(DEV), x["beta"].to(DEV), sd)
+        assert o.dtype == torch.float16
+        ro, ref = oracle_decode_heads(x, ref, DECODE_HEADS)
+        eo, mo = _max_err(o, ro, sel)
+        worst_o = max(worst_o, eo)
+        _gate(f"step {step} o", eo, mo, w.tol_o)
+    es, ms = _max_err(sd, ref, sel)
+    print(f"f16 decode 1000 steps: worst o err {worst_o:.3e}, state err {es:.3e} (max|S| {ms:.3e})")
+    _gate("state", es, ms, w.tol_state)
+
+
+def test_decode_b1_step_captured_once_and_replayed_1000_times():
+    """One request at a time (the pages' serving regime): the decode step of one
+    sequence (16 q/k, 32 value heads, d=128) is captured once in a CUDA graph
+    that reads fixed input buffers, and replayed 1000 times, each time after
+    that step's fresh tokens are copied into those buffers. o is compared with
+    the oracle at every step (every head) and the state after the last one."""
+    B, Hqk, Hv, d, steps = 1, 16, 32, 128, 1000
+    names = ("q", "k", "v", "g", "beta")
+    xs = [workloads.decode_step_inputs(s, B, Hqk, Hv, d) for s in range(steps)]
+    staged = {n: torch.stack([x[n] for x in xs]).to(DEV) for n in names}   # [steps, ...] on the device
+    fixed = {n: torch.empty_like(staged[n][0]) for n in names}
+    state = workloads.decode_state(B, Hv, d, std=0.05)
+    ref = state.double().numpy().copy()
+    sd = state.to(DEV)
+    o_fixed = torch.empty(B, Hv, d, dtype=torch.bfloat16, device=DEV)
+    o_all = torch.full((steps, B, Hv, d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):   # warm-up outside capture (first launch of the kernel)
+        for n in names:
+            fixed[n].copy_(staged[n][0])
+        probe = sd.clone()
+        gdn.decode(*(fixed[n] for n in names), probe, o=o_fixed)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        gdn.decode(*(fixed[n] for n in names), sd, o=o_fixed)
+    for s in range(steps):
+        for n in names:
+            fixed[n].copy_(staged[n][s])
+        graph.replay()
+        o_all[s].copy_(o_fixed)
+    torch.cuda.synchronize()
+    gdn.device_error()
+    worst = 0.0
+    for s in range(steps):
+        ro, ref = oracle.decode(xs[s]["q"], xs[s]["k"], xs[s]["v"], xs[s]["g"], xs[s]["beta"], ref)
+        eo, mo = _max_err(o_all[s], ro)
+        worst = max(worst, eo)
+        _gate(f"step {s} o", eo, mo, 2e-2)
+    es, ms = _max_err(sd, ref)
+    print(f"B=1 graph-replayed decode, 1000 steps: worst o err {worst:.3e}, state err {es:.3e}")
+    _gate("state", es, ms, 1e-2)
+
+
+def test_decode_back_to_back_launches_read_the_previous_state():
+    """Consecutive decode steps on one stream with nothing between them, each
+    reading the state the previous one wrote: 200 steps of 64 sequences x 32
+    heads must equal the oracle's sequential steps."""
+    B, Hqk, Hv, d, steps = 64, 16, 32, 128, 200
+    heads = [0, 31]
+    state = workloads.decode_state(B, Hv, d, std=0.05)
+    ref = state.double().numpy().copy()
+    sd = state.to(DEV)
+    xs = [workloads.decode_step_inputs(s, B, Hqk, Hv, d) for s in range(steps)]
+    staged = [{n: x[n].to(DEV) for n in ("q", "k", "v", "g", "beta")} for x in xs]
+    torch.cuda.synchronize()
+    outs = [gdn.decode(x["q"], x["k"], x["v"], x["g"], x["beta"], sd) for x in staged]
+    torch.cuda.synchronize()
+    for s in range(steps):
+        ro, ref = oracle_decode_heads(xs[s], ref, heads)
+        eo, mo = _max_err(outs[s], ro, (slice(None), heads))
+        _gate(f"step {s} o", eo, mo, 2e-2)
+    es, ms = _max_err(sd, ref, (slice(None), heads))
+    _gate("state", es, ms, 1e-2)
+
+
 def test_decode_workload_1000_steps_sampled_heads():
     """64 sequences x 32 value heads, d=128, 1000 consecutive steps; o checked at
     every step and the state after the last one, on value heads 0, 13 and 31."""
@@ -214,10 +305,10 @@ def test_prefill_small_bf16_ragged(lengths):
 
 
 @pytest.mark.parametrize("d", [16, 32, 64])
-@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16, torch.float32])
 def test_prefill_small_heads_simt(d, dtype):
     x = workloads.prefill_inputs([50, 17], Hqk=1, Hv=2, d=d, dtype=dtype, seed=91 + d, state_std=0.05)
-    tol = 2e-2 if dtype == torch.bfloat16 else 1e-4
+    tol = 2e-2 if dtype != torch.float32 else 1e-4
     for chunk in (16, 32, 64):
         check_prefill(x, tol, tol if dtype == torch.float32 else 1e-2, chunk=chunk)
 
@@ -247,6 +338,30 @@ def test_prefill_workload_qwen08b_layer_full():
     """1 x 4096 tokens, 16 q/k and 16 v heads, d=128, bf16: every element."""
     w = workloads.workload("prefill")
     check_prefill(workloads.inputs_for(w), w.tol_o, w.tol_state)
+
+
+def test_prefill_workload_qwen08b_layer_full_f16():
+    """The same layer with f16 inputs and output (the pages' second numerical
+    mode: 16-bit data, f32 accumulation): every element against the unchanged
+    oracle, at the bf16 tolerances."""
+    w = workloads.workload("prefill", dtype="f16")
+    x = workloads.inputs_for(w)
+    assert x["q"].dtype == torch.float16
+    eo, es = check_prefill(x, w.tol_o, w.tol_state)
+    print(f"f16 layer: o err {eo:.3e}, state err {es:.3e}")
+
+
+@pytest.mark.parametrize("lengths", [[1], [65], [197], [5, 130, 1, 64, 77]])
+def test_prefill_small_f16_ragged(lengths):
+    x = workloads.prefill_inputs(lengths, Hqk=2, Hv=4, d=128, dtype=torch.float16, seed=177 + sum(lengths),
+                                 state_std=0.05)
+    check_prefill(x, 2e-2, 1e-2)
+
+
+def test_prefill_long_f16_sampled_heads():
+    """The 32768-token prompt (16 q/k, 32 value heads) with f16 inputs."""
+    w = workloads.workload("long", dtype="f16")
+    check_prefill(workloads.inputs_for(w), w.tol_o, w.tol_state, heads=[0, 17, 31])
 
 
 @pytest.mark.parametrize("T,heads", [(32768, [0, 9, 18, 31]), (81920, [0, 13, 31])])

@@ -49,7 +49,7 @@ class Workload:
     Hqk: int = 16
     Hv: int = 16
     d: int = 128
-    dtype: str = "bf16"        # dtype of q, k, v, o ("bf16" or "f32")
+    dtype: str = "bf16"        # dtype of q, k, v, o ("bf16", "f16" or "f32")
     chunk: int = 64
     state_std: float = 0.0     # 0 => zero initial state
     tol_o: float = 2e-2        # max abs error vs the fp64 oracle
@@ -61,7 +61,7 @@ class Workload:
 
     @property
     def torch_dtype(self):
-        return torch.bfloat16 if self.dtype == "bf16" else torch.float32
+        return {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}[self.dtype]
 
 
 def varlen_lengths(n: int = 8, lo: int = 128, hi: int = 8192, seed: int = SEED_VARLEN_LENGTHS):
@@ -69,8 +69,17 @@ def varlen_lengths(n: int = 8, lo: int = 128, hi: int = 8192, seed: int = SEED_V
     return [int(x) for x in torch.randint(lo, hi + 1, (n,), generator=g)]
 
 
-def workload(name: str, T: int | None = None) -> Workload:
-    """The named workload; ``T`` overrides the length of single-sequence prefill."""
+def workload(name: str, T: int | None = None, dtype: str | None = None) -> Workload:
+    """The named workload; ``T`` overrides the length of single-sequence prefill
+    and ``dtype`` the input type of a 16-bit workload ("f16": the same draws
+    rounded to IEEE half instead of bfloat16)."""
+    w = _workload(name, T)
+    if dtype is not None:
+        w.dtype = dtype
+    return w
+
+
+def _workload(name: str, T: int | None = None) -> Workload:
     if name == "tiny":
         return Workload("tiny", 0, "prefill", lengths=[64], Hqk=2, Hv=2, d=16,
                         dtype="f32", chunk=16, tol_o=1e-4, tol_state=1e-4)
@@ -136,7 +145,8 @@ def prefill_inputs(lengths, Hqk, Hv, d, dtype=torch.bfloat16, seed=SEED_TOKENS +
 
 
 def decode_step_inputs(step, B, Hqk, Hv, d, dtype=torch.bfloat16, dv=None):
-    """Inputs of decode step ``step`` (fresh seeded tokens each step)."""
+    """Inputs of decode step ``step`` (fresh seeded tokens each step); q, k, v
+    are drawn in fp32 and rounded to ``dtype`` (bf16, f16, or kept fp32)."""
     dv = dv or d
     gen = torch.Generator().manual_seed(SEED_DECODE_STEP + step)
     q = torch.randn(B, Hqk, d, generator=gen).to(dtype)
