@@ -43,17 +43,17 @@
 //              time and run only the state chain on the packages, k and v.
 //
 // Every CTA has eight compute warps (0-7) and three with jobs of their own.
-// Warps 8 and 9 do what waits on other CTAs or on memory, a step ahead: in a
-// chain CTA warp 8 acquires ready flags and issues the copies of package, k
-// and v, and warp 9 hands ring slots back once a copy has landed; in a prep
-// CTA warp 8 claims items, fetches their gates and tiles and waits for ring
-// slots, and warp 9 publishes finished packages. In a chain CTA warp 10 issues
-// every tensor-core product, so the compute warps only run the epilogues (U_s
-// on warps 0, 1, 4, 5, O on 2, 3, 6, 7, which also store O; then the state);
-// in a prep CTA warp 0 issues the MMAs and warp 10 is idle. Handovers use
-// mbarriers with bounded waits; compute warps synchronise among themselves
-// with named barrier 1 (and the four O warps of a chain CTA with barrier 2). (The register file is allocated per 128 threads, so
-// eleven warps cost no registers over nine.)
+// In a chain CTA warp 8 acquires ready flags and issues the copies of package,
+// k and v, warp 9 hands ring slots back once a copy has landed, and warp 10
+// issues every tensor-core product, so the compute warps only run the
+// epilogues (U_s on warps 0, 1, 4, 5, O on 2, 3, 6, 7, which also store O;
+// then the state). Y and dS commit to barriers of their own and every compute
+// warp waits for them on its own. In a prep CTA warp 8 claims items, fetches
+// their gates and tiles and waits for ring slots, warp 9 publishes finished
+// packages and warp 0 of the compute warps issues the MMAs. Handovers use
+// mbarriers with bounded waits; the prep compute warps synchronise among
+// themselves with named barrier 1. (The register file is allocated per 128
+// threads, so eleven warps cost no registers over nine.)
 //
 // Ring protocol. The chain CTAs work on the slice-chains in rounds; in round r
 // chain j = r P + q runs at position q < P (P chains per round). Each position
@@ -96,6 +96,7 @@ constexpr int kRelWarp = 9;          // chain: hands ring slots back; prep: publ
 constexpr int kMmaWarp = 10;         // chain: issues the tensor-core work
 constexpr uint32_t kTmemCols = 512;
 constexpr int kRing = 12;            // package slots per ring position
+constexpr int kFlagStride = 32;      // flag words per ring position: each position's flags on a 128-byte line
 constexpr int kMaxRounds = 1024;
 constexpr int kMaxPositions = 74;    // chains per round at most
 
@@ -110,9 +111,9 @@ constexpr uint32_t kPkgStride = 50176;
 // ---- workspace layout ----
 struct Workspace {
   static constexpr size_t kCounter = 0;      // uint32 counter of the items after the first one per prep CTA
-  static constexpr size_t kFlags = 256;      // ready[positions][R], then consumed[positions][R]
+  static constexpr size_t kFlags = 256;      // ready[positions][32], then consumed[positions][32] (R used)
   __host__ __device__ static constexpr size_t flags_bytes(long positions) {
-    return (size_t)positions * kRing * 2 * sizeof(uint32_t);
+    return (size_t)positions * kFlagStride * 2 * sizeof(uint32_t);
   }
   __host__ __device__ static constexpr size_t pkg_offset(long positions) {
     return (kFlags + flags_bytes(positions) + 1023) & ~size_t(1023);
@@ -124,15 +125,18 @@ struct Workspace {
 };
 
 // ---- TMEM column map ----
-constexpr uint32_t kColG = 0;      // prep: [k;q] k^T       M=128, N=64
-constexpr uint32_t kColN = 64;     // prep: N = D A_o       M=64 (lanes 0-15)
-constexpr uint32_t kColS2 = 128;   // prep: N D (lanes 0-15), N^2 (lanes 16-31)
-constexpr uint32_t kColZ = 192;    // prep: N^2 E           M=64
-constexpr uint32_t kColW = 256;    // prep: -W, d_k 0-63 in lanes 0-15, 64-127 in lanes 16-31
-constexpr uint32_t kColPW = 320;   // prep: -P W, the same split
-constexpr uint32_t kColPT = 384;   // prep: P T_u           M=64, N=64 (lanes 0-15)
-constexpr uint32_t kColY = 0;      // chain: Y = [U ; O]    M=128, N=DVP, two buffers 128 columns apart
-constexpr uint32_t kColDS = 256;   // chain: dS^T           M=128, N=DVP
+// prep: a stage's accumulator is read out before the next stage's MMA is
+// issued, so later stages reuse the columns of earlier ones
+constexpr uint32_t kColG = 0;      // [k;q] k^T             M=128, N=64
+constexpr uint32_t kColN = 64;     // N = D A_o             M=64 (lanes 0-15)
+constexpr uint32_t kColS2 = 128;   // N D (lanes 0-15), N^2 (lanes 16-31)
+constexpr uint32_t kColZ = 0;      // N^2 E                 M=64 (the Gram columns, read in stage 1)
+constexpr uint32_t kColW = 64;     // -W, d_k 0-63 in lanes 0-15, 64-127 in lanes 16-31 (N's columns)
+constexpr uint32_t kColPW = 128;   // -P W, the same split (N D, N^2's columns)
+constexpr uint32_t kColPT = 192;   // P T_u                 M=64, N=64 (lanes 0-15)
+// chain:
+constexpr uint32_t kColY = 0;      // Y = [U ; O]           M=128, N=DVP, two buffers 128 columns apart
+constexpr uint32_t kColDS = 256;   // dS^T                  M=128, N=DVP
 
 template <int DVP>
 struct Smem {
@@ -142,12 +146,14 @@ struct Smem {
   static constexpr int kBlocks = DVP / kBlk;
   static constexpr uint32_t kRB = kBlk * 2;
   static constexpr uint32_t kR = DVP * 2;
-  // chain role: two input buffers {package image, k tile, v slice}
+  // chain role: kNB input buffers {package image, k tile, v slice} (three, where
+  // they fit at 32-row slices, measured no faster than two)
+  static constexpr int kNB = 2;
   static constexpr uint32_t kIn = 0;
   static constexpr uint32_t kInK = kPkgStride;                // k [64][128] as two 64-column halves, 8 KB apart
   static constexpr uint32_t kInV = kInK + 16384;              // v [64][DVP]
   static constexpr uint32_t kInBytes = (kInV + 64 * kR + 1023) & ~1023u;
-  static constexpr uint32_t kUsb = 2 * kInBytes;              // U_s [64][DVP]
+  static constexpr uint32_t kUsb = kNB * kInBytes;            // U_s [64][DVP]
   static constexpr uint32_t kSb = kUsb + ((64 * kR + 1023) & ~1023u);   // S^T [128][DVP]
   static constexpr uint32_t kChainEnd = kSb + 128 * kR;
   // prep role (aliases the chain region; a CTA has one role)
@@ -173,8 +179,8 @@ struct Smem {
   static constexpr uint32_t kPrepEnd = kRBase + 4 * (kMaxRounds + 1);
   // common
   static constexpr uint32_t kCommon = ((kChainEnd > kPrepEnd ? kChainEnd : kPrepEnd) + 7) & ~7u;
-  static constexpr uint32_t kBarA = kCommon;                  // full[2], free[2], mma, pub[2] | u, o, s
-  static constexpr uint32_t kMisc = kBarA + 8 * 8;            // tmem slot, scan[4]
+  static constexpr uint32_t kBarA = kCommon;                  // mbarriers (chain 9, prep 16)
+  static constexpr uint32_t kMisc = kBarA + 16 * 8;           // tmem slot, scan[4]
   static constexpr uint32_t kTotal = kMisc + 64;
   static constexpr uint32_t kAlloc = kTotal + 1024;
   static_assert(kAlloc <= 227 * 1024, "shared memory budget");
@@ -241,12 +247,15 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
   const uint32_t sbase = smem_u32(sm);
   int* round_start = reinterpret_cast<int*>(sm + L::kRounds);
   int* rbase = reinterpret_cast<int*>(sm + L::kRBase);
-  uint64_t* bar_full = reinterpret_cast<uint64_t*>(sm + L::kBarA);  // [2] control -> compute
-  uint64_t* bar_free = bar_full + 2;                                 // [2] compute -> control
-  uint64_t* bar_mma = bar_full + 4;
-  uint64_t* bar_pub = bar_full + 5;                                  // [2] prep: publisher -> hand-over
-  uint64_t* bar_u = bar_full + 5;      // chain: U_s staged (the 4 U warps)
-  uint64_t* bar_s = bar_full + 7;      // chain: the 16-bit state copy is written
+  // chain-role mbarriers (the prep role's sixteen are named where it starts)
+  constexpr int NB = L::kNB;
+  uint64_t* bar_full = reinterpret_cast<uint64_t*>(sm + L::kBarA);  // [NB] input buffer landed
+  uint64_t* bar_free = bar_full + NB;                                // [NB] input buffer free again
+  uint64_t* bar_mma = bar_full + 2 * NB;   // the Y product's commits
+  uint64_t* bar_u = bar_mma + 1;           // U_s staged (the 4 U warps)
+  uint64_t* bar_ds = bar_mma + 2;          // the dS product's commits
+  uint64_t* bar_s = bar_mma + 3;           // the 16-bit state copy is written (the 8 compute warps)
+  uint64_t* bar_o = bar_mma + 4;           // O staged for the TMA store (the 4 O warps)
   uint32_t* misc = reinterpret_cast<uint32_t*>(sm + L::kMisc);     // [0] tmem, [2..5] scan
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -264,7 +273,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
 
   uint32_t* counter = reinterpret_cast<uint32_t*>(p.ws + Workspace::kCounter);
   uint32_t* ready = reinterpret_cast<uint32_t*>(p.ws + Workspace::kFlags);   // [position][slot]
-  uint32_t* consumed = ready + (long)chains_per_round * kRing;
+  uint32_t* consumed = ready + (long)chains_per_round * kFlagStride;
   uint8_t* pkgs = p.ws + Workspace::pkg_offset(chains_per_round);
 
   auto seq_bounds = [&](int n, int& tb, int& te) {
@@ -282,12 +291,18 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     // it and the releasing warp has seen its copy land (so that the releasing warp,
     // which waits by parity, never falls a phase behind); U_s and O are staged by
     // four warps each
-    for (int i = 0; i < 8; ++i) {
-      uint32_t count = 1;
-      if (is_chain && (i == 2 || i == 3)) count = 9;   // free: the 8 compute warps + the releasing warp
-      if (is_chain && i == 5) count = 4;               // U_s staged: the 4 U warps
-      if (is_chain && i == 7) count = 8;               // state copy written: the 8 compute warps
-      mbar_init(&bar_full[i], count);
+    if (is_chain) {
+      for (int i = 0; i < NB; ++i) {
+        mbar_init(&bar_full[i], 1);
+        mbar_init(&bar_free[i], 9);   // the 8 compute warps + the releasing warp
+      }
+      mbar_init(bar_mma, 1);
+      mbar_init(bar_u, 4);            // the 4 U warps
+      mbar_init(bar_ds, 1);
+      mbar_init(bar_s, 8);            // the 8 compute warps
+      mbar_init(bar_o, 4);            // the 4 O warps
+    } else {
+      for (int i = 0; i < 16; ++i) mbar_init(&bar_full[i], 1);
     }
     fence_mbar_init();
     prefetch_tensormap(&qmap);
@@ -307,29 +322,12 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
   const uint32_t tmem = misc[0];
   const uint32_t tlane = static_cast<uint32_t>(qd * 32) << 16;
 
-  // compute-warp barriers (named barrier 1 over warps 0-7)
-  auto cbar = [&]() { named_bar_sync(1, kCompute); };
-  auto cbar_and = [&](bool ok) { return named_bar_and(1, kCompute, ok); };
-  uint32_t mma_phase = 0;
   bool abort = false;
-  auto wait_mma = [&](bool also_ok = true) -> bool {
-    bool ok = mbar_wait(bar_mma, mma_phase) && also_ok;
-    mma_phase ^= 1;
-    ok = cbar_and(ok);
-    tc_fence_after();
-    return ok;
-  };
-  auto publish = [&]() {   // shared-memory writes -> visible to the tensor core; TMEM reads done
-    fence_async_smem();
-    tc_fence_before();
-    cbar();
-    tc_fence_after();
-  };
 
   if (is_chain) {
     // ============================== chain role ==============================
     // The CTA runs slice-chains sc = blockIdx.x + r NC in turn; input buffer
-    // gc & 1 holds the gc-th chunk it runs (package, k tile, v slice).
+    // gc % NB holds the gc-th chunk it runs (package, k tile, v slice).
     auto decode_sc = [&](long sc, long& j, int& h, int& i0, int& t_begin, int& t_end) {
       j = sc / kSlices;
       h = (int)(j % Hv);
@@ -349,7 +347,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     if (is_ctl) {
       // ---- issuing warp: per chunk, wait for the package's ready flag and a free input
       //      buffer, then copy package, k and v in ----
-      const uint32_t* rdy = ready + q * kRing;
+      const uint32_t* rdy = ready + q * kFlagStride;
       const uint8_t* ring = pkgs + (size_t)q * kRing * kPkgStride;
       long gc = 0;
       int base = 0;
@@ -366,13 +364,13 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           break;
         }
         for (int c = 0; c < nch; ++c, ++gc) {
-          const int b = (int)(gc & 1);
+          const int b = (int)(gc % NB);
           const int s = base + c, slot = s % kRing;
           if (!GDN_CHECK(s >= 0 && t_begin + c * kC < t_end)) { abort = true; break; }
           bool ok = true;
           if (lane == 0) ok = wait_flag_geq(&rdy[slot], (uint32_t)(s / kRing + 1));
           if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) { abort = true; break; }
-          if (gc >= 2 && !mbar_wait(&bar_free[b], (uint32_t)((gc - 2) >> 1) & 1u)) { abort = true; break; }
+          if (gc >= NB && !mbar_wait(&bar_free[b], (uint32_t)((gc - NB) / NB) & 1u)) { abort = true; break; }
           __syncwarp();
           fence_async_global();
           uint8_t* dst = sm + L::kIn + b * L::kInBytes;
@@ -390,7 +388,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     } else if (is_rel) {
       // ---- releasing warp: hands each ring slot back once its copy has landed, and
       //      counts the numbers a shorter chain leaves unused as read ----
-      uint32_t* cns = consumed + q * kRing;
+      uint32_t* cns = consumed + q * kFlagStride;
       long gc = 0;
       int base = 0;
       for (long sc = blockIdx.x; sc < n_slice_chains && !abort; sc += NC) {
@@ -401,10 +399,10 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         const int maxc = round_maxc(j, q);
         if (!GDN_CHECK(q < chains_per_round && base >= 0 && maxc >= nch)) { abort = true; break; }
         for (int c = 0; c < nch; ++c, ++gc) {
-          if (!mbar_wait(&bar_full[gc & 1], (uint32_t)(gc >> 1) & 1u)) { abort = true; break; }
+          if (!mbar_wait(&bar_full[gc % NB], (uint32_t)(gc / NB) & 1u)) { abort = true; break; }
           __syncwarp();
           if (lane == 0) {
-            mbar_arrive(&bar_free[gc & 1]);   // (the buffer is not refilled before this)
+            mbar_arrive(&bar_free[gc % NB]);   // (the buffer is not refilled before this)
             red_add_release_gpu(&cns[(base + c) % kRing], 1u);
           }
         }
@@ -425,10 +423,8 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         //      warps through mbarriers (bounded) ----
         auto issue_a2v = [&](int b, uint32_t ycol) {   // A2 V_raw of input buffer b, the first term of Y
           const uint32_t in = sbase + L::kIn + b * L::kInBytes;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_f16_warp(tmem + ycol, desc_kmajor(in + kPkgA2, kk, 0), desc_mnmajor(in + L::kInV, kk, kRB, 64 * kRB),
-                          kIdY, kk > 0);
+          mma_k<4, true, 0, false, kRB>(tmem + ycol, desc_kmajor(in + kPkgA2, 0, 0),
+                                        desc_mnmajor(in + L::kInV, 0, kRB, 64 * kRB), kIdY, false);
         };
         long gc = 0;
         bool early = false;
@@ -439,37 +435,34 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           decode_sc(sc, j, h, i0, t_begin, t_end);
           const int nch = (t_end - t_begin + kC - 1) / kC;
           for (int c = 0; c < nch; ++c, ++gc) {
-            const int b = (int)(gc & 1);
+            const int b = (int)(gc % NB);
             const uint32_t in = sbase + L::kIn + b * L::kInBytes;
-            const uint32_t ycol = kColY + 128u * (uint32_t)b;
-            if (!mbar_wait(&bar_full[b], (uint32_t)(gc >> 1) & 1u) || !mbar_wait(bar_s, ph_s)) { abort = true; break; }
+            const uint32_t ycol = kColY + 128u * (uint32_t)(gc & 1);   // two Y buffers in TMEM
+            if (!mbar_wait(&bar_full[b], (uint32_t)(gc / NB) & 1u) || !mbar_wait(bar_s, ph_s)) { abort = true; break; }
             ph_s ^= 1;
             __syncwarp();
             tc_fence_after();
             if (!early) issue_a2v(b, ycol);
-            if (c > 0 || p.state_in != nullptr) {   // (a first chunk from a zero state has no A1 S^T;
-#pragma unroll                                        //  its package carries no A1)
-              for (int kk = 0; kk < 8; ++kk)
-                mma_f16_warp(tmem + ycol, desc_kmajor(in + kPkgA1, kk, 16384), desc_mnmajor(sSb, kk, kRB, 128 * kRB),
-                              kIdY, 1u);
-            }
+            if (c > 0 || p.state_in != nullptr)   // (a first chunk from a zero state has no A1 S^T;
+                                                  //  its package carries no A1)
+              mma_k<8, true, 16384, false, kRB>(tmem + ycol, desc_kmajor(in + kPkgA1, 0, 16384),
+                                                desc_mnmajor(sSb, 0, kRB, 128 * kRB), kIdY, true);
             mma_commit_warp(bar_mma);
             if (!mbar_wait(bar_u, ph_u)) { abort = true; break; }
             ph_u ^= 1;
             __syncwarp();
             tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_f16_warp(tmem + kColDS, desc_mnmajor(in + L::kInK, kk, 128, 8192),
-                            desc_mnmajor(sUsb, kk, kRB, 64 * kRB), kIdDS, kk > 0);
-            mma_commit_warp(bar_mma);
+            mma_k<4, false, 128, false, kRB>(tmem + kColDS, desc_mnmajor(in + L::kInK, 0, 128, 8192),
+                                             desc_mnmajor(sUsb, 0, kRB, 64 * kRB), kIdDS, false);
+            mma_commit_warp(bar_ds);
             // the other Y buffer was last read in chunk gc - 1, whose epilogues all ended
             // before the compute warps' state update of that chunk (and so before bar_u)
             early = false;
             if (c + 1 < nch) {
-              const bool nxt = mbar_test_wait(&bar_full[b ^ 1], (uint32_t)((gc + 1) >> 1) & 1u);
+              const int bn = (int)((gc + 1) % NB);
+              const bool nxt = mbar_test_wait(&bar_full[bn], (uint32_t)((gc + 1) / NB) & 1u);
               if (__shfl_sync(0xffffffffu, nxt ? 1 : 0, 0)) {
-                issue_a2v(b ^ 1, kColY + 128u * (uint32_t)(b ^ 1));
+                issue_a2v(bn, kColY + 128u * (uint32_t)((gc + 1) & 1));
                 early = true;
               }
             }
@@ -477,7 +470,14 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         }
       } else {
         // ---- compute warps: the Y and dS epilogues and the fp32 state ----
+        // Every warp waits for the products on its own: Y and dS commit to separate
+        // barriers, and neither product of the next chunk can complete before every
+        // warp has arrived after reading this one (bar_s), so no warp can miss a
+        // phase. The O warps meet on an mbarrier before the TMA store. No wait here
+        // is unbounded: a warp whose wait runs out stops, and the others' waits
+        // then run out in turn.
         long gc = 0;
+        uint32_t ph_y = 0, ph_ds = 0, ph_o = 0;
         auto warp_arrive = [&](uint64_t* bar) {
           __syncwarp();
           if (lane == 0) mbar_arrive(bar);
@@ -510,21 +510,26 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           }
 
           for (int c = 0; c < nch; ++c, ++gc) {
-            const int b = (int)(gc & 1);
+            const int b = (int)(gc % NB);
+            const uint32_t yb = (uint32_t)(gc & 1);   // the Y buffer in TMEM
             const uint32_t in = sbase + L::kIn + b * L::kInBytes;
             const uint8_t* in_g = sm + L::kIn + b * L::kInBytes;
-            const bool full_ok = mbar_wait(&bar_full[b], (uint32_t)(gc >> 1) & 1u);
             const int len = min(kC, t_end - (t_begin + c * kC));
             const bool o_tma = len == kC;
             if (!GDN_CHECK(len > 0 && t_begin + c * kC + len <= p.total_T)) { abort = true; break; }
-            if (!wait_mma(full_ok)) { abort = true; break; }   // Y
+            if (!mbar_wait(&bar_full[b], (uint32_t)(gc / NB) & 1u) || !mbar_wait(bar_mma, ph_y)) {   // Y
+              abort = true;
+              break;
+            }
+            ph_y ^= 1;
+            tc_fence_after();
             {
               const float us = qd < 2 ? reinterpret_cast<const float*>(in_g + kPkgUs)[r128] : 0.f;
               T* orow = out + ((size_t)(t_begin + c * kC + (r128 & 63)) * Hv + h) * kD + i0 + ch * kHalf;
 #pragma unroll
               for (int pp = 0; pp < kHalf / kPart; ++pp) {
                 float yv[kPart];
-                tmem_ld<kPart>(tmem + tlane + kColY + 128u * (uint32_t)b + ch * kHalf + pp * kPart, yv);
+                tmem_ld<kPart>(tmem + tlane + kColY + 128u * yb + ch * kHalf + pp * kPart, yv);
                 if (qd < 2) {   // U_s = diag(us) U -> shared memory (T) for dS
 #pragma unroll
                   for (int q2 = 0; q2 < kPart; ++q2) yv[q2] *= us;
@@ -547,16 +552,25 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             tc_fence_before();
             if (qd < 2) {
               warp_arrive(bar_u);
-            } else if (o_tma) {   // the O warps meet, then thread 64 stores the O tile
-              named_bar_sync(2, 128);
+            } else if (o_tma) {   // the O warps' staging is complete, then thread 64 stores the O tile
+              warp_arrive(bar_o);
               if (tid == 64) {
+                if (!mbar_wait(bar_o, ph_o)) {
+                  abort = true;
+                } else {
 #pragma unroll
-                for (int vb = 0; vb < L::kBlocks; ++vb)
-                  tma_store_3d(&omap, in_g + L::kInV + vb * 64 * kRB, i0 + vb * L::kBlk, h, t_begin + c * kC);
-                bulk_commit_group();
+                  for (int vb = 0; vb < L::kBlocks; ++vb)
+                    tma_store_3d(&omap, in_g + L::kInV + vb * 64 * kRB, i0 + vb * L::kBlk, h, t_begin + c * kC);
+                  bulk_commit_group();
+                }
               }
+              ph_o ^= 1;
+              abort = __shfl_sync(0xffffffffu, abort ? 1 : 0, 0) != 0;   // (warp-uniform)
+              if (abort) break;
             }
-            if (!wait_mma()) { abort = true; break; }   // dS
+            if (!mbar_wait(bar_ds, ph_ds)) { abort = true; break; }   // dS
+            ph_ds ^= 1;
+            tc_fence_after();
             {
               const float gL = *reinterpret_cast<const float*>(in_g + kPkgGL);
 #pragma unroll
@@ -616,6 +630,43 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     __syncthreads();
     const int total_items = round_start[n_rounds];
 
+    // prep-role mbarriers: a two-entry queue between the hand-over warp and the
+    // compute warps, the compute warps' MMA commits, the publisher's hand-back
+    uint64_t* bar_pfull = bar_full;        // [2] hand-over -> compute: entry k & 1 (its tiles counted in bytes)
+    uint64_t* bar_pfree = bar_full + 2;    // [2] compute -> publisher: the package copies are complete
+    uint64_t* bar_pmma = bar_full + 4;     // the compute warps' MMA commits
+    uint64_t* bar_ppub = bar_full + 5;     // [2] publisher -> hand-over: the entry may be reused
+    // compute-warp barriers (named barrier 1 over warps 0-7)
+    auto cbar = [&]() { named_bar_sync(1, kCompute); };
+    auto cbar_and = [&](bool ok) { return named_bar_and(1, kCompute, ok); };
+    uint32_t mma_phase = 0;
+    // wait for an MMA commit with the compute warps' barrier (which also makes
+    // the result consistent across them), or without it when the next barrier,
+    // publish(ok), takes the decision: every MMA of the next stage is issued
+    // after that barrier, so no thread can miss a phase of bar_pmma
+    auto wait_mma = [&](bool also_ok = true) -> bool {
+      bool ok = mbar_wait(bar_pmma, mma_phase) && also_ok;
+      mma_phase ^= 1;
+      ok = cbar_and(ok);
+      tc_fence_after();
+      return ok;
+    };
+    auto wait_mma_local = [&]() -> bool {
+      const bool ok = mbar_wait(bar_pmma, mma_phase);
+      mma_phase ^= 1;
+      tc_fence_after();
+      return ok;
+    };
+    // shared-memory writes -> visible to the tensor core; TMEM reads done; returns
+    // whether `ok` holds on every compute thread
+    auto publish = [&](bool ok) -> bool {
+      fence_async_smem();
+      tc_fence_before();
+      ok = cbar_and(ok);
+      tc_fence_after();
+      return ok;
+    };
+
     if (is_ctl) {
       // ---- hand-over warp: claim items, fetch gates and raw k, q tiles, wait for the
       //      ring slot and hand the item over; queue entry k & 1 is reused once the
@@ -672,11 +723,11 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             v = 0;
           }
           uint8_t* kq = sm + L::kKQP + b * 32768;
-          mbar_expect_tx_warp(&bar_full[b], 4 * 8192);
-          tma_load_3d_warp(kq, &kmap, &bar_full[b], 0, hq, c0);
-          tma_load_3d_warp(kq + 16384, &kmap, &bar_full[b], 64, hq, c0);
-          tma_load_3d_warp(kq + 8192, &qmap, &bar_full[b], 0, hq, c0);
-          tma_load_3d_warp(kq + 16384 + 8192, &qmap, &bar_full[b], 64, hq, c0);
+          mbar_expect_tx_warp(&bar_pfull[b], 4 * 8192);
+          tma_load_3d_warp(kq, &kmap, &bar_pfull[b], 0, hq, c0);
+          tma_load_3d_warp(kq + 16384, &kmap, &bar_pfull[b], 64, hq, c0);
+          tma_load_3d_warp(kq + 8192, &qmap, &bar_pfull[b], 0, hq, c0);
+          tma_load_3d_warp(kq + 16384 + 8192, &qmap, &bar_pfull[b], 64, hq, c0);
           float* qg = reinterpret_cast<float*>(qe + 16);
           float* qb = reinterpret_cast<float*>(qe + 80);
 #pragma unroll
@@ -685,7 +736,8 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             qb[e] = e < len ? p.beta[(size_t)(c0 + e) * Hv + h] : 0.f;
           }
           // (numbers below kRing have no previous occupant to wait for)
-          if (lane == 0 && s >= kRing) ok = wait_flag_geq(&consumed[q * kRing + s % kRing], (uint32_t)(kSlices * (s / kRing)));
+          if (lane == 0 && s >= kRing)
+            ok = wait_flag_geq(&consumed[q * kFlagStride + s % kRing], (uint32_t)(kSlices * (s / kRing)));
           ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         }
         const bool go = v && ok && len > 0;
@@ -699,11 +751,11 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         __syncwarp();
         // the arrival publishes the entry; the phase completes once the tiles are in too
         // (an item that gave up after starting its tiles still lets them land first)
-        if (lane == 0) mbar_arrive(&bar_full[b]);
+        if (lane == 0) mbar_arrive(&bar_pfull[b]);
         return go;
       };
       for (int k = 0;; ++k) {
-        if (k >= 2 && !mbar_wait(&bar_pub[k & 1], (uint32_t)((k - 2) >> 1) & 1u)) break;
+        if (k >= 2 && !mbar_wait(&bar_ppub[k & 1], (uint32_t)((k - 2) >> 1) & 1u)) break;
         __syncwarp();
         if (!hand_over(k)) break;
       }
@@ -713,14 +765,14 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       for (int it = 0;; ++it) {
         const int b = it & 1;
         const uint32_t par = (uint32_t)(it >> 1) & 1u;
-        if (!mbar_wait(&bar_full[b], par)) break;   // handed over (or the end marker)
+        if (!mbar_wait(&bar_pfull[b], par)) break;   // handed over (or the end marker)
         const uint32_t* qe = reinterpret_cast<const uint32_t*>(sm + L::kQueue + b * L::kQueueBytes);
         if (qe[0] == 0) break;
         if (!GDN_CHECK(qe[2] < (uint32_t)chains_per_round)) break;
-        if (!mbar_wait(&bar_free[b], par)) break;
-        if (lane == 0) st_release_gpu(&ready[qe[2] * kRing + qe[1] % kRing], qe[1] / kRing + 1);
+        if (!mbar_wait(&bar_pfree[b], par)) break;
+        if (lane == 0) st_release_gpu(&ready[qe[2] * kFlagStride + qe[1] % kRing], qe[1] / kRing + 1);
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar_pub[b]);
+        if (lane == 0) mbar_arrive(&bar_ppub[b]);
       }
     } else if (warp < 8) {
       // ---- compute warps (warp 10 has no job in a prep CTA) ----
@@ -746,7 +798,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         if (out_pending < 0) return;
         bulk_wait_all();
         fence_async_global();
-        mbar_arrive(&bar_free[out_pending]);
+        mbar_arrive(&bar_pfree[out_pending]);
         out_pending = -1;
       };
       for (int it = 0; !abort; ++it) {
@@ -754,10 +806,10 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         const uint32_t* qe = reinterpret_cast<const uint32_t*>(sm + L::kQueue + b * L::kQueueBytes);
         // The previous package is published during this item's first stage, unless
         // this item is not here yet: its ring slot may wait for that package.
-        if (tid == kOutThread && out_pending >= 0 && !mbar_test_wait(&bar_full[b], (uint32_t)(it >> 1) & 1u))
+        if (tid == kOutThread && out_pending >= 0 && !mbar_test_wait(&bar_pfull[b], (uint32_t)(it >> 1) & 1u))
           finish_out();
         {
-          const bool w = mbar_wait(&bar_full[b], (uint32_t)(it >> 1) & 1u);
+          const bool w = mbar_wait(&bar_pfull[b], (uint32_t)(it >> 1) & 1u);
           if (!cbar_and(w)) { abort = true; break; }
         }
         if (qe[0] == 0) break;
@@ -775,10 +827,9 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
 
         // ---- Gram [k;q] k^T on the tensor core; gates scan and norms meanwhile ----
         if (warp == 0) {
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_f16_warp(tmem + kColG, desc_kmajor(sKQ, kk, 16384), desc_kmajor(sKQ, kk, 16384), kIdG, kk > 0);
-          mma_commit_warp(bar_mma);
+          mma_k<8, true, 16384, true, 16384>(tmem + kColG, desc_kmajor(sKQ, 0, 16384), desc_kmajor(sKQ, 0, 16384),
+                                             kIdG, false);
+          mma_commit_warp(bar_pmma);
         } else if (tid == kOutThread) {
           finish_out();   // (before this item's vectors reuse the staging)
         }
@@ -932,17 +983,15 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             st_shared_v4(sbase + L::kDm + sw128_off(row, 8 * cc, 0), make_uint4(0, 0, 0, 0));
           }
         }
-        publish();
+        publish(true);
 
         // ---- N = D A_o ----
         if (warp == 0) {
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_f16_warp(tmem + kColN, desc_kmajor(sbase + L::kDm, kk, 0), desc_mnmajor(sbase + L::kAo, kk, 128, 8192),
-                          kId64, kk > 0);
-          mma_commit_warp(bar_mma);
+          mma_k<4, true, 0, false, 128>(tmem + kColN, desc_kmajor(sbase + L::kDm, 0, 0),
+                                        desc_mnmajor(sbase + L::kAo, 0, 128, 8192), kId64, false);
+          mma_commit_warp(bar_pmma);
         }
-        if (!wait_mma()) { abort = true; break; }
+        const bool ok_n = wait_mma_local();
         {
           float v[32];
           tmem_ld32(tmem + tlane + kColN + 32 * ch, v);
@@ -952,21 +1001,17 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
               st_shared_v4(sbase + L::kNm + sw128_off(r64, 32 * ch + 8 * c8, 0), pack8<T>(v + 8 * c8));
           }
         }
-        publish();
+        if (!publish(ok_n)) { abort = true; break; }
 
         // ---- N D (lanes 0-15) and N^2 (lanes 16-31) ----
         if (warp == 0) {
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_f16_warp(tmem + kColS2, desc_kmajor(sbase + L::kNm, kk, 0),
-                          desc_mnmajor(sbase + L::kDm, kk, 128, 8192), kId64, kk > 0);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_f16_warp(tmem + (16u << 16) + kColS2, desc_kmajor(sbase + L::kNm, kk, 0),
-                          desc_mnmajor(sbase + L::kNm, kk, 128, 8192), kId64, kk > 0);
-          mma_commit_warp(bar_mma);
+          const uint64_t nm = desc_kmajor(sbase + L::kNm, 0, 0);
+          mma_k<4, true, 0, false, 128>(tmem + kColS2, nm, desc_mnmajor(sbase + L::kDm, 0, 128, 8192), kId64, false);
+          mma_k<4, true, 0, false, 128>(tmem + (16u << 16) + kColS2, nm, desc_mnmajor(sbase + L::kNm, 0, 128, 8192),
+                                        kId64, false);
+          mma_commit_warp(bar_pmma);
         }
-        if (!wait_mma()) { abort = true; break; }
+        const bool ok_s2 = wait_mma_local();
         float E[32];   // lanes 0-15: columns 32ch..32ch+31 of row r64 of E = D - N D (fp32)
         {
           float v[32];
@@ -986,17 +1031,15 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
               st_shared_v4(sbase + L::kN2 + sw128_off(r64, 32 * ch + 8 * c8, 0), pack8<T>(v + 8 * c8));
           }
         }
-        publish();
+        if (!publish(ok_s2)) { abort = true; break; }
 
         // ---- Z = N^2 E ; T = E + Z -> T_u (shared and package), -T_w (shared) ----
         if (warp == 0) {
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_f16_warp(tmem + kColZ, desc_kmajor(sbase + L::kN2, kk, 0), desc_mnmajor(sbase + L::kEm, kk, 128, 8192),
-                          kId64, kk > 0);
-          mma_commit_warp(bar_mma);
+          mma_k<4, true, 0, false, 128>(tmem + kColZ, desc_kmajor(sbase + L::kN2, 0, 0),
+                                        desc_mnmajor(sbase + L::kEm, 0, 128, 8192), kId64, false);
+          mma_commit_warp(bar_pmma);
         }
-        if (!wait_mma()) { abort = true; break; }
+        const bool ok_z = wait_mma_local();
         {
           float z[32];
           tmem_ld32(tmem + tlane + kColZ + 32 * ch, z);
@@ -1017,24 +1060,20 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             }
           }
         }
-        publish();
+        if (!publish(ok_z)) { abort = true; break; }
 
         // ---- -W = (-T_w) K_raw -> shared (operand of P W and A1 rows 0-63); the two
         //      column halves go to the two lane halves so that every thread has work ----
         const int dhalf = 64 * (lane >> 4) + 32 * ch;   // this thread's 32 columns of a d_k-wide row
         if (need_a1) {
           if (warp == 0) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_f16_warp(tmem + kColW, desc_kmajor(sbase + L::kTw, kk, 0), desc_mnmajor(sKQ, kk, 128, 16384), kId64,
-                            kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_f16_warp(tmem + (16u << 16) + kColW, desc_kmajor(sbase + L::kTw, kk, 0),
-                            desc_mnmajor(sKQ + 16384, kk, 128, 16384), kId64, kk > 0);
-            mma_commit_warp(bar_mma);
+            const uint64_t tw = desc_kmajor(sbase + L::kTw, 0, 0);
+            mma_k<4, true, 0, false, 128>(tmem + kColW, tw, desc_mnmajor(sKQ, 0, 128, 16384), kId64, false);
+            mma_k<4, true, 0, false, 128>(tmem + (16u << 16) + kColW, tw, desc_mnmajor(sKQ + 16384, 0, 128, 16384),
+                                          kId64, false);
+            mma_commit_warp(bar_pmma);
           }
-          if (!wait_mma()) { abort = true; break; }
+          const bool ok_w = wait_mma_local();
           {
             float w[32];
             tmem_ld32(tmem + tlane + kColW + 32 * ch, w);
@@ -1042,28 +1081,22 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             for (int c8 = 0; c8 < 4; ++c8)
               st_shared_v4(sbase + L::kWm + sw128_off(r64, dhalf + 8 * c8, 8192), pack8<T>(w + 8 * c8));
           }
-          publish();
+          if (!publish(ok_w)) { abort = true; break; }
         }
 
         // ---- -P W and P T_u -> A1 rows 64-127 = rho Q_raw - P W, A2 rows 64-127 = P T_u ----
         if (warp == 0) {
           if (need_a1) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_f16_warp(tmem + kColPW, desc_kmajor(sbase + L::kPm, kk, 0),
-                            desc_mnmajor(sbase + L::kWm, kk, 128, 8192), kId64, kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_f16_warp(tmem + (16u << 16) + kColPW, desc_kmajor(sbase + L::kPm, kk, 0),
-                            desc_mnmajor(sbase + L::kWm + 8192, kk, 128, 8192), kId64, kk > 0);
+            mma_k<4, true, 0, false, 128>(tmem + kColPW, desc_kmajor(sbase + L::kPm, 0, 0),
+                                          desc_mnmajor(sbase + L::kWm, 0, 128, 8192), kId64, false);
+            mma_k<4, true, 0, false, 128>(tmem + (16u << 16) + kColPW, desc_kmajor(sbase + L::kPm, 0, 0),
+                                          desc_mnmajor(sbase + L::kWm + 8192, 0, 128, 8192), kId64, false);
           }
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_f16_warp(tmem + kColPT, desc_kmajor(sbase + L::kPm, kk, 0), desc_mnmajor(sbase + L::kTu, kk, 128, 8192),
-                          kId64, kk > 0);
-          mma_commit_warp(bar_mma);
+          mma_k<4, true, 0, false, 128>(tmem + kColPT, desc_kmajor(sbase + L::kPm, 0, 0),
+                                        desc_mnmajor(sbase + L::kTu, 0, 128, 8192), kId64, false);
+          mma_commit_warp(bar_pmma);
         }
-        if (!wait_mma()) { abort = true; break; }
+        const bool ok_pw = wait_mma_local();
         {
           const float rho = vRho[r64];
           if (need_a1) {
@@ -1089,10 +1122,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         }
         // ---- the package images are complete: copy them out in bulk; the copies are
         //      waited for during the next item, then the control warp publishes ----
-        fence_async_smem();
-        tc_fence_before();
-        cbar();
-        tc_fence_after();
+        if (!publish(ok_pw)) { abort = true; break; }
         if (tid == kOutThread) {   // (a CTA's first package is published at once: chains are starting)
           if (need_a1) {
             bulk_store(pkg + kPkgA1, sm + L::kWm, 8192);

@@ -330,6 +330,36 @@ __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t base, int kk, uint32_t
   return smem_desc(base + kk * 16 * row_bytes, lbo, 8 * row_bytes, sw);
 }
 
+// Byte offset of K-step kk (16 elements) within a K-major 128B-swizzled
+// operand whose 64-element atom columns are `acs` bytes apart, and within an
+// MN-major operand with K-rows of `row_bytes`.
+__host__ __device__ constexpr uint32_t kmajor_step(int kk, uint32_t acs) {
+  return static_cast<uint32_t>(kk >> 2) * acs + static_cast<uint32_t>(kk & 3) * 32u;
+}
+__host__ __device__ constexpr uint32_t mnmajor_step(int kk, uint32_t row_bytes) {
+  return static_cast<uint32_t>(kk) * 16u * row_bytes;
+}
+// A descriptor with its start address moved on by `bytes` (a multiple of 16).
+// The 14-bit address field cannot carry into the next one: shared-memory
+// addresses stay below 256 KB.
+__device__ __forceinline__ uint64_t desc_advance(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+
+// NK K-steps of D (+)= A B (kind::f16), issued by the whole warp (one elected
+// lane), from descriptors a0, b0 of K-step 0 built once: each later step only
+// advances their start addresses by constants. A_KM / B_KM say whether the
+// operand is K-major (then A_P / B_P is its atom column spacing) or MN-major
+// (then the byte length of its K-rows). acc: accumulate onto D from the first
+// step on (else the first step overwrites D).
+template <int NK, bool A_KM, uint32_t A_P, bool B_KM, uint32_t B_P>
+__device__ __forceinline__ void mma_k(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint32_t idesc, bool acc) {
+#pragma unroll
+  for (int kk = 0; kk < NK; ++kk) {
+    const uint32_t ao = A_KM ? kmajor_step(kk, A_P) : mnmajor_step(kk, A_P);
+    const uint32_t bo = B_KM ? kmajor_step(kk, B_P) : mnmajor_step(kk, B_P);
+    mma_f16_warp(d_tmem, desc_advance(a0, ao), desc_advance(b0, bo), idesc, (acc || kk > 0) ? 1u : 0u);
+  }
+}
+
 // Byte offset of element (row, col) in a K-major 128B-swizzled operand
 // (64-element atom columns `acs` bytes apart). col % 8 == 0 addresses a chunk.
 __device__ __forceinline__ uint32_t sw128_off(int row, int col, uint32_t acs) {

@@ -171,21 +171,22 @@ class MBarrier:
         return (self.phase & 1) != parity
 
 
-def chain_cta_run(n_chunks, rng, releasing_warp_arrives=True, max_idle=5000):
-    """The issuing, releasing and compute warps of one chain CTA over two input
-    buffers. A copy lands some time after it is issued (completing bar_full); the
-    releasing warp counts each landed copy once; compute reads each chunk in
+def chain_cta_run(n_chunks, rng, releasing_warp_arrives=True, max_idle=5000, nb=2):
+    """The issuing, releasing and compute warps of one chain CTA over nb input
+    buffers (chunk gc in buffer gc % nb, its use number gc // nb giving the
+    parity). A copy lands some time after it is issued (completing bar_full);
+    the releasing warp counts each landed copy once; compute reads each chunk in
     order. Returns the chunks the releasing warp counted."""
-    full = [MBarrier(1), MBarrier(1)]
-    free = [MBarrier(2 if releasing_warp_arrives else 1) for _ in range(2)]
+    full = [MBarrier(1) for _ in range(nb)]
+    free = [MBarrier(2 if releasing_warp_arrives else 1) for _ in range(nb)]
     in_flight = []            # buffers whose copy has been issued but has not landed
     counted = []
 
     def issuer():
         for gc in range(n_chunks):
-            b = gc & 1
-            if gc >= 2:
-                while not free[b].test_wait(((gc - 2) >> 1) & 1):
+            b = gc % nb
+            if gc >= nb:
+                while not free[b].test_wait(((gc - nb) // nb) & 1):
                     yield "wait"
             in_flight.append(b)
             yield "step"
@@ -202,8 +203,8 @@ def chain_cta_run(n_chunks, rng, releasing_warp_arrives=True, max_idle=5000):
 
     def releaser():
         for gc in range(n_chunks):
-            b = gc & 1
-            while not full[b].test_wait((gc >> 1) & 1):
+            b = gc % nb
+            while not full[b].test_wait((gc // nb) & 1):
                 yield "wait"
             if releasing_warp_arrives:
                 free[b].arrive()
@@ -212,8 +213,8 @@ def chain_cta_run(n_chunks, rng, releasing_warp_arrives=True, max_idle=5000):
 
     def compute():
         for gc in range(n_chunks):
-            b = gc & 1
-            while not full[b].test_wait((gc >> 1) & 1):
+            b = gc % nb
+            while not full[b].test_wait((gc // nb) & 1):
                 yield "wait"
             for _ in range(rng.randint(0, 3)):   # the chunk's work
                 yield "step"
@@ -238,9 +239,10 @@ def chain_cta_run(n_chunks, rng, releasing_warp_arrives=True, max_idle=5000):
     return counted
 
 
-def test_chain_cta_releasing_warp_never_loses_a_phase():
+@pytest.mark.parametrize("nb", [2, 3])
+def test_chain_cta_releasing_warp_never_loses_a_phase(nb):
     for seed in range(200):
-        assert chain_cta_run(24, random.Random(seed)) == list(range(24))
+        assert chain_cta_run(24, random.Random(seed), nb=nb) == list(range(24))
 
 
 def test_a_releasing_warp_that_does_not_gate_the_buffer_can_lose_a_phase():
@@ -357,19 +359,25 @@ def test_publication_held_until_the_next_item_deadlocks_on_a_small_ring():
 
 # ------------------------------ a chain CTA's MMA warp and compute warps ---
 
-def chain_mma_run(n_chunks, rng, max_idle=5000):
-    """The MMA warp and the compute warps of one chain CTA (the compute warps
-    move together: their waits end in a barrier across all eight). Per chunk the
-    MMA warp waits for the input and for the bf16 state copy (bar_s), issues Y and
-    commits it to bar_mma, waits for U_s (bar_u), issues dS and commits it to the
-    same bar_mma; a commit completes when its products finish, some time later.
-    The compute warps wait for Y on bar_mma, stage U_s (bar_u), wait for dS on
-    bar_mma, update the state and write its copy (bar_s). Every wait is by
-    parity. Returns the (chunk, product) pairs the compute warps read."""
-    mma, bar_u, bar_s = MBarrier(1), MBarrier(1), MBarrier(1)
+def chain_mma_run(n_chunks, rng, max_idle=5000, separate_barriers=True):
+    """The MMA warp and the eight compute warps of one chain CTA, each warp an
+    agent of its own (no barrier across them). Per chunk the MMA warp waits for
+    the 16-bit state copy of all eight warps (bar_s), issues Y and commits it,
+    waits for U_s from the four U warps (bar_u), issues dS and commits it. With
+    separate_barriers, Y commits to bar_y and dS to bar_ds; otherwise both to one
+    barrier (the planted mistake for per-warp waits). A commit completes when its
+    product finishes, some time later, in issue order. Each compute warp waits
+    for Y, then (U warps) arrives on bar_u or (O warps) on bar_o, where the first
+    O warp waits for all four before its store; then it waits for dS and arrives
+    on bar_s. Every wait is by parity. Returns each warp's reads as (chunk,
+    product, the latest completed product of that kind when it read)."""
+    bar_y, bar_ds = MBarrier(1), MBarrier(1)
+    if not separate_barriers:
+        bar_ds = bar_y
+    bar_u, bar_s, bar_o = MBarrier(4), MBarrier(8), MBarrier(4)
     issued = []               # products whose commit has not completed yet
-    done = []                 # products completed, in order
-    seen = []
+    last = {}                 # kind -> the latest completed product
+    seen = {w: [] for w in range(8)}
 
     def mma_warp():
         ph_s = ph_u = 0
@@ -385,36 +393,46 @@ def chain_mma_run(n_chunks, rng, max_idle=5000):
             issued.append((gc, "dS"))
             yield "step"
 
-    def tensor_core():        # commits complete in order, each a while after its issue
+    def tensor_core():
         n = 0
         while n < 2 * n_chunks:
             if issued and rng.random() < 0.4:
-                done.append(issued.pop(0))
-                mma.arrive()
+                gc, kind = issued.pop(0)
+                last[kind] = gc
+                (bar_y if kind == "Y" else bar_ds).arrive()
                 n += 1
                 yield "step"
             else:
                 yield "wait"
 
-    def compute():
-        ph = 0
+    def compute(w):
+        u_warp = w in (0, 1, 4, 5)
+        ph_y = ph_ds = ph_o = 0
         bar_s.arrive()        # the first state copy
         for gc in range(n_chunks):
-            while not mma.test_wait(ph):
+            while not bar_y.test_wait(ph_y):
                 yield "wait"
-            ph ^= 1
-            seen.append((gc, "Y", done[-1] if done else None))
-            bar_u.arrive()
+            ph_y ^= 1
+            seen[w].append((gc, "Y", last.get("Y")))
             yield "step"
-            while not mma.test_wait(ph):
+            if u_warp:
+                bar_u.arrive()
+            else:
+                bar_o.arrive()
+                if w == 2:    # the storing O warp waits for the other three
+                    while not bar_o.test_wait(ph_o):
+                        yield "wait"
+                ph_o ^= 1
+            yield "step"
+            while not bar_ds.test_wait(ph_ds):
                 yield "wait"
-            ph ^= 1
-            seen.append((gc, "dS", done[-1] if done else None))
+            ph_ds ^= 1
+            seen[w].append((gc, "dS", last.get("dS")))
             if gc + 1 < n_chunks:
                 bar_s.arrive()
             yield "step"
 
-    live = [mma_warp(), tensor_core(), compute()]
+    live = [mma_warp(), tensor_core()] + [compute(w) for w in range(8)]
     idle = 0
     while live:
         a = rng.choice(live)
@@ -430,12 +448,33 @@ def chain_mma_run(n_chunks, rng, max_idle=5000):
     return seen
 
 
-def test_chain_mma_handshake_reads_each_product_once_in_order():
-    """Y and dS share one barrier: the compute warps must see each completion as
-    the product they wait for -- the MMA warp cannot commit the next product
-    before they have seen the last, since it waits on them in between."""
+def test_chain_mma_handshake_each_warp_reads_each_product_once_in_order():
+    """Y and dS on their own barriers, compute warps waiting independently: every
+    warp sees each product as the latest completed one of its kind -- the next
+    product of a kind cannot complete before every warp has arrived after reading
+    this one -- and nothing hangs."""
     for seed in range(200):
         seen = chain_mma_run(12, random.Random(seed))
-        assert [(g, p) for g, p, _ in seen] == [(g, p) for g in range(12) for p in ("Y", "dS")]
-        for g, p, last_done in seen:
-            assert last_done == (g, p), "a later product completed before this one was read"
+        for w in range(8):
+            assert [(g, p) for g, p, _ in seen[w]] == [(g, p) for g in range(12) for p in ("Y", "dS")]
+            for g, p, latest in seen[w]:
+                assert latest == g, f"warp {w} read {p} of chunk {g} when chunk {latest}'s had completed"
+
+
+def test_one_shared_commit_barrier_lets_a_lagging_warp_read_the_wrong_product():
+    """With Y and dS on one barrier and no barrier across the compute warps, a
+    warp that lags reads a later completion as the one it waits for (or waits
+    for a phase that has come round again): the model must notice."""
+    bad = 0
+    for seed in range(300):
+        try:
+            seen = chain_mma_run(12, random.Random(seed), separate_barriers=False)
+        except AssertionError:
+            bad += 1
+            continue
+        for w in range(8):
+            if [(g, p) for g, p, _ in seen[w]] != [(g, p) for g in range(12) for p in ("Y", "dS")] or \
+                    any(latest != g for g, p, latest in seen[w]):
+                bad += 1
+                break
+    assert bad > 0

@@ -177,3 +177,33 @@ def test_device_runner_applies_the_plan_times_and_fills_fresh_outputs(monkeypatc
     # and the whole selection through the device leg
     best, results = tune.tune_prefill(q, k, v, g, beta, None, cu, plans=[(32, 16), (128, 4)], reps=2)
     assert all(r.ok for r in results) and (best.dvp, best.nc) == (32, 16)
+
+
+@pytest.mark.gpu
+def test_tune_prefill_on_the_device_returns_a_gated_plan_that_matches_the_oracle():
+    """The tuner's whole device leg on a B200: two 700-token sequences, 4 q/k and
+    8 value heads. Every candidate plan is timed and gated against the default
+    plan; the chosen plan must have passed, and its output must also match the
+    fp64 oracle at the bf16 prefill tolerances and the 1/64 rule."""
+    import numpy as np
+
+    import gated_deltanet_linear_21_b200 as gdn
+    import oracle
+    import workloads
+
+    x = workloads.prefill_inputs([700, 700], Hqk=4, Hv=8, d=128, seed=8800, state_std=0.05)
+    d = {kk: (vv.to("cuda") if isinstance(vv, torch.Tensor) else vv) for kk, vv in x.items()}
+    args = (d["q"], d["k"], d["v"], d["g"], d["beta"], d["state_in"], d["cu_seqlens"])
+    best, results = tune.tune_prefill(*args, reps=3)
+    assert best.ok and math.isfinite(best.ms) and best.ms > 0
+    assert len(results) >= 3 and all(r.ok for r in results), [r.reason for r in results if not r.ok]
+    o, s = gdn.prefill(*args, plan=(best.dvp, best.nc))
+    o_def, s_def = gdn.prefill(*args)
+    torch.cuda.synchronize()
+    gdn.device_error()
+    ro, rs = oracle.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], x["state_in"], x["cu_seqlens"])
+    for got, ref, tol in ((o, ro, 2e-2), (s, rs, 1e-2), (o_def, ro, 2e-2), (s_def, rs, 1e-2)):
+        a = got.double().cpu().numpy()
+        err = float(np.abs(a - ref).max())
+        assert err <= tol and err <= np.abs(ref).max() / 64
+    print("plans:", [(r.dvp, r.nc, round(r.ms, 4), f"{r.err:.1e}") for r in results], "best", (best.dvp, best.nc))
