@@ -137,6 +137,7 @@ constexpr uint32_t kColPT = 192;   // P T_u                 M=64, N=64 (lanes 0-
 // chain:
 constexpr uint32_t kColY = 0;      // Y = [U ; O]           M=128, N=DVP, two buffers 128 columns apart
 constexpr uint32_t kColDS = 256;   // dS^T                  M=128, N=DVP
+constexpr uint32_t kColA1 = 384;   // A1 staged as the A operand of A1 S^T: two buffers of 64 columns
 
 template <int DVP>
 struct Smem {
@@ -417,7 +418,8 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       const uint32_t sSb = sbase + L::kSb;
       const uint32_t sUsb = sbase + L::kUsb;
       if (warp == kMmaWarp) {
-        // ---- MMA warp: per chunk Y = A2 V + A1 S^T (rows 0-63 U, rows 64-127 O) into
+        // ---- MMA warp: per chunk Y = A2 V + A1 S^T (rows 0-63 U, rows 64-127 O; A1 staged
+        //      in TMEM by tcgen05.cp, so that only S^T streams from shared memory) into
         //      TMEM buffer gc & 1, then dS^T = K_raw^T U_s and, when the next chunk's
         //      data is in, its A2 V into the other Y buffer; it waits on the compute
         //      warps through mbarriers (bounded) ----
@@ -425,6 +427,14 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           const uint32_t in = sbase + L::kIn + b * L::kInBytes;
           mma_k<4, true, 0, false, kRB>(tmem + ycol, desc_kmajor(in + kPkgA2, 0, 0),
                                         desc_mnmajor(in + L::kInV, 0, kRB, 64 * kRB), kIdY, false);
+        };
+        // the package's A1 (input buffer b) into TMEM buffer ab, so that A1 S^T reads
+        // only S^T from shared memory on the chain (the copy is ordered before it)
+        auto stage_a1 = [&](int b, uint32_t ab) {
+          const uint64_t a0 = desc_kmajor(sbase + L::kIn + b * L::kInBytes + kPkgA1, 0, 16384);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            tmem_cp_128x256b_warp(tmem + kColA1 + 64u * ab + 8u * kk, desc_advance(a0, kmajor_step(kk, 16384)));
         };
         long gc = 0;
         bool early = false;
@@ -442,11 +452,20 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             ph_s ^= 1;
             __syncwarp();
             tc_fence_after();
+            const uint32_t ab = (uint32_t)(gc & 1);   // the A1 buffer in TMEM
             if (!early) issue_a2v(b, ycol);
-            if (c > 0 || p.state_in != nullptr)   // (a first chunk from a zero state has no A1 S^T;
-                                                  //  its package carries no A1)
-              mma_k<8, true, 16384, false, kRB>(tmem + ycol, desc_kmajor(in + kPkgA1, 0, 16384),
-                                                desc_mnmajor(sSb, 0, kRB, 128 * kRB), kIdY, true);
+            if (c > 0 || p.state_in != nullptr) {   // (a first chunk from a zero state has no A1 S^T;
+                                                    //  its package carries no A1)
+              const uint64_t s0 = desc_mnmajor(sSb, 0, kRB, 128 * kRB);
+              if (early) {   // A1 was staged in TMEM while the previous chunk ran
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                  mma_f16_tmem_a_warp(tmem + ycol, tmem + kColA1 + 64u * ab + 8u * kk,
+                                      desc_advance(s0, mnmajor_step(kk, kRB)), kIdY, 1u);
+              } else {       // staging it now would only add a pass: read it from shared memory
+                mma_k<8, true, 16384, false, kRB>(tmem + ycol, desc_kmajor(in + kPkgA1, 0, 16384), s0, kIdY, true);
+              }
+            }
             mma_commit_warp(bar_mma);
             if (!mbar_wait(bar_u, ph_u)) { abort = true; break; }
             ph_u ^= 1;
@@ -456,13 +475,16 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
                                              desc_mnmajor(sUsb, 0, kRB, 64 * kRB), kIdDS, false);
             mma_commit_warp(bar_ds);
             // the other Y buffer was last read in chunk gc - 1, whose epilogues all ended
-            // before the compute warps' state update of that chunk (and so before bar_u)
+            // before the compute warps' state update of that chunk (and so before bar_u);
+            // the other A1 buffer was last read by chunk gc - 1's Y product, complete
+            // before its U_s epilogue
             early = false;
             if (c + 1 < nch) {
               const int bn = (int)((gc + 1) % NB);
               const bool nxt = mbar_test_wait(&bar_full[bn], (uint32_t)((gc + 1) / NB) & 1u);
               if (__shfl_sync(0xffffffffu, nxt ? 1 : 0, 0)) {
                 issue_a2v(bn, kColY + 128u * (uint32_t)((gc + 1) & 1));
+                stage_a1(bn, (uint32_t)((gc + 1) & 1));   // (a later chunk of a chain always has A1)
                 early = true;
               }
             }
