@@ -382,7 +382,8 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           tma_load_3d_warp(dst + L::kInK + 8192, &kmap, &bar_full[b], 64, hq, c0);
 #pragma unroll
           for (int vb = 0; vb < L::kBlocks; ++vb)
-            tma_load_3d_warp(dst + L::kInV + vb * 64 * L::kRB, &vmap, &bar_full[b], i0 + vb * L::kBlk, h, c0);
+            tma_load_3d_warp_hint(dst + L::kInV + vb * 64 * L::kRB, &vmap, &bar_full[b], i0 + vb * L::kBlk, h, c0,
+                                  l2_evict_first_policy());   // (its only reader)
         }
         base += maxc;
       }
@@ -519,7 +520,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           }
           float Sreg[kHalf];
 #pragma unroll
-          for (int q2 = 0; q2 < kHalf; ++q2) Sreg[q2] = p.state_in ? p.state_in[s_off + (size_t)q2 * kD] : 0.f;
+          for (int q2 = 0; q2 < kHalf; ++q2) Sreg[q2] = p.state_in ? __ldcs(p.state_in + s_off + (size_t)q2 * kD) : 0.f;
           auto store_state = [&]() {
 #pragma unroll
             for (int c8 = 0; c8 < kHalf / 8; ++c8)
@@ -582,7 +583,8 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
                 } else {
 #pragma unroll
                   for (int vb = 0; vb < L::kBlocks; ++vb)
-                    tma_store_3d(&omap, in_g + L::kInV + vb * 64 * kRB, i0 + vb * L::kBlk, h, t_begin + c * kC);
+                    tma_store_3d_hint(&omap, in_g + L::kInV + vb * 64 * kRB, i0 + vb * L::kBlk, h, t_begin + c * kC,
+                                      l2_evict_first_policy());
                   bulk_commit_group();
                 }
               }
@@ -617,7 +619,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           }
           if (abort) break;
 #pragma unroll
-          for (int q2 = 0; q2 < kHalf; ++q2) p.state_out[s_off + (size_t)q2 * kD] = Sreg[q2];
+          for (int q2 = 0; q2 < kHalf; ++q2) __stcs(p.state_out + s_off + (size_t)q2 * kD, Sreg[q2]);
         }
       }
     }
