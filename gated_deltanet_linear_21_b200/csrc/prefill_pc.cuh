@@ -49,8 +49,9 @@
 // epilogues (U_s on warps 0, 1, 4, 5, O on 2, 3, 6, 7, which also store O;
 // then the state). Y and dS commit to barriers of their own and every compute
 // warp waits for them on its own. In a prep CTA warp 8 claims items, fetches
-// their gates and tiles and waits for ring slots, warp 9 publishes finished
-// packages and warp 0 of the compute warps issues the MMAs. Handovers use
+// their gates and tiles and waits for ring slots, warp 10 copies each staged
+// package out to its ring slot and publishes it once the copies are complete,
+// and warp 0 of the compute warps issues the MMAs (warp 9 has no job there). Handovers use
 // mbarriers with bounded waits; the prep compute warps synchronise among
 // themselves with named barrier 1. (The register file is allocated per 128
 // threads, so eleven warps cost no registers over nine.)
@@ -61,9 +62,9 @@
 // base_r the sum over earlier rounds of the longest chain's chunk count; slot
 // s mod R holds package s. The prep hand-over warp waits until consumed[q][s mod R]
 // >= slices * (s / R) (every slice read the previous occupant) before it hands
-// the item over; the compute warps stage the package in shared memory and copy
-// it out with bulk copies, and once those are complete (and fenced) the
-// publishing warp sets ready[q][s mod R] = s / R + 1 with release semantics. A
+// the item over; the compute warps stage the package in shared memory, the
+// writing warp copies it out with bulk copies and, once those are complete (and
+// fenced), sets ready[q][s mod R] = s / R + 1 with release semantics. A
 // chain's issuing warp waits for that value with acquire semantics and copies
 // the package into shared memory; its releasing warp then adds 1 to
 // consumed[q][s mod R] (and arrives on the input buffer's free barrier, so that
@@ -170,7 +171,7 @@ struct Smem {
   static constexpr uint32_t kWm = kTu + 8192;                 // -W [64][128], two halves 8 KB apart
   static constexpr uint32_t kA1b = kWm + 16384;               // rho Q - P W [64][128], two halves 8 KB apart
   static constexpr uint32_t kA2b = kA1b + 16384;              // P T_u [64][64]
-  static constexpr uint32_t kPv = kA2b + 8192;                // package vectors: us[64], gamma_L, tokens
+  static constexpr uint32_t kPv = kA2b + 8192;                // package vectors: us[64], gamma_L, tokens (2 x 512 B)
   static constexpr uint32_t kAd = kPv + 1024;                 // diagonal blocks of A, fp32 [4][16][16]
   static constexpr uint32_t kVec = kAd + 4096;                // 8 vectors of 64 fp32
   static constexpr uint32_t kQueue = kVec + 8 * 256;          // 2 items handed over by the control warp:
@@ -655,11 +656,13 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     const int total_items = round_start[n_rounds];
 
     // prep-role mbarriers: a two-entry queue between the hand-over warp and the
-    // compute warps, the compute warps' MMA commits, the publisher's hand-back
+    // compute warps, the compute warps' MMA commits, and the hand-offs of a
+    // package from the compute warps to the writing warp, and back
     uint64_t* bar_pfull = bar_full;        // [2] hand-over -> compute: entry k & 1 (its tiles counted in bytes)
-    uint64_t* bar_pfree = bar_full + 2;    // [2] compute -> publisher: the package copies are complete
     uint64_t* bar_pmma = bar_full + 4;     // the compute warps' MMA commits
-    uint64_t* bar_ppub = bar_full + 5;     // [2] publisher -> hand-over: the entry may be reused
+    uint64_t* bar_ppub = bar_full + 5;     // [2] writer -> hand-over: published, the entry may be reused
+    uint64_t* bar_pstage = bar_full + 7;   // [2] compute -> writer: the package images are staged
+    uint64_t* bar_psread = bar_full + 9;   // [2] writer -> compute: the staged images have been read
     // compute-warp barriers (named barrier 1 over warps 0-7)
     auto cbar = [&]() { named_bar_sync(1, kCompute); };
     auto cbar_and = [&](bool ok) { return named_bar_and(1, kCompute, ok); };
@@ -694,7 +697,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     if (is_ctl) {
       // ---- hand-over warp: claim items, fetch gates and raw k, q tiles, wait for the
       //      ring slot and hand the item over; queue entry k & 1 is reused once the
-      //      publishing warp has published item k - 2 ----
+      //      writing warp has published item k - 2 ----
       auto hand_over = [&](int k) -> bool {   // false once none is left (or a wait ran out)
         const int b = k & 1;
         uint32_t* qe = reinterpret_cast<uint32_t*>(sm + L::kQueue + b * L::kQueueBytes);
@@ -783,9 +786,12 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         __syncwarp();
         if (!hand_over(k)) break;
       }
-    } else if (is_rel) {
-      // ---- publishing warp: once the compute warps have written item `it`'s package
-      //      (their bulk copies complete and fenced), release its ready flag ----
+    } else if (warp == kMmaWarp) {
+      // ---- writing warp: copies each package the compute warps have staged out to its
+      //      ring slot in bulk, tells them once the images have been read (they are
+      //      overwritten from the next item's T stage on), and once the copies are
+      //      complete (and ordered before it) releases the package's ready flag and
+      //      hands the queue entry back ----
       for (int it = 0;; ++it) {
         const int b = it & 1;
         const uint32_t par = (uint32_t)(it >> 1) & 1u;
@@ -793,13 +799,32 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         const uint32_t* qe = reinterpret_cast<const uint32_t*>(sm + L::kQueue + b * L::kQueueBytes);
         if (qe[0] == 0) break;
         if (!GDN_CHECK(qe[2] < (uint32_t)chains_per_round)) break;
-        if (!mbar_wait(&bar_pfree[b], par)) break;
-        if (lane == 0) st_release_gpu(&ready[qe[2] * kFlagStride + qe[1] % kRing], qe[1] / kRing + 1);
+        if (!mbar_wait(&bar_pstage[b], par)) break;
+        // (a chain's first chunk from a zero state carries no A1)
+        const bool need_a1 = qe[4] != 0 || p.state_in != nullptr;
+        uint8_t* pkg = pkgs + ((size_t)qe[2] * kRing + qe[1] % kRing) * kPkgStride;
+        if (lane == 0) {
+          if (need_a1) {
+            bulk_store(pkg + kPkgA1, sm + L::kWm, 8192);
+            bulk_store(pkg + kPkgA1 + 16384, sm + L::kWm + 8192, 8192);
+            bulk_store(pkg + kPkgA1 + 8192, sm + L::kA1b, 8192);
+            bulk_store(pkg + kPkgA1 + 16384 + 8192, sm + L::kA1b + 8192, 8192);
+          }
+          bulk_store(pkg + kPkgA2, sm + L::kTu, 8192);
+          bulk_store(pkg + kPkgA2 + 8192, sm + L::kA2b, 8192);
+          bulk_store(pkg + kPkgUs, sm + L::kPv + 512 * b, kPkgCopy - kPkgUs);
+          bulk_commit_group();
+          bulk_wait_read_all();
+          mbar_arrive(&bar_psread[b]);
+          bulk_wait_all();
+          fence_async_global();
+          st_release_gpu(&ready[qe[2] * kFlagStride + qe[1] % kRing], qe[1] / kRing + 1);
+          mbar_arrive(&bar_ppub[b]);
+        }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar_ppub[b]);
       }
     } else if (warp < 8) {
-      // ---- compute warps (warp 10 has no job in a prep CTA) ----
+      // ---- compute warps ----
       constexpr uint32_t kIdG = idesc_f16kind(128, 64, false, false, kFmt);
       constexpr uint32_t kId64 = idesc_f16kind(64, 64, false, true, kFmt);
       float* vG = reinterpret_cast<float*>(sm + L::kVec);   // per-warp partial scan of g
@@ -813,25 +838,9 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       float* Ad = reinterpret_cast<float*>(sm + L::kAd);
       float* scan = reinterpret_cast<float*>(&misc[2]);
 
-      // Thread 32 (warp 1, idle while the Gram product runs) owns the package's bulk
-      // copies: once those of the previous package are complete, it orders them
-      // before the publishing warp's release and hands the item back.
-      constexpr int kOutThread = 32;
-      int out_pending = -1;
-      auto finish_out = [&]() {
-        if (out_pending < 0) return;
-        bulk_wait_all();
-        fence_async_global();
-        mbar_arrive(&bar_pfree[out_pending]);
-        out_pending = -1;
-      };
       for (int it = 0; !abort; ++it) {
         const int b = it & 1;
         const uint32_t* qe = reinterpret_cast<const uint32_t*>(sm + L::kQueue + b * L::kQueueBytes);
-        // The previous package is published during this item's first stage, unless
-        // this item is not here yet: its ring slot may wait for that package.
-        if (tid == kOutThread && out_pending >= 0 && !mbar_test_wait(&bar_pfull[b], (uint32_t)(it >> 1) & 1u))
-          finish_out();
         {
           const bool w = mbar_wait(&bar_pfull[b], (uint32_t)(it >> 1) & 1u);
           if (!cbar_and(w)) { abort = true; break; }
@@ -846,7 +855,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
 #endif
         // a chain's first chunk from a zero state never multiplies A1 (S = 0): skip -W, P W
         const bool need_a1 = qe[4] != 0 || p.state_in != nullptr;
-        uint8_t* pkg = pkgs + ((size_t)qe[2] * kRing + qe[1] % kRing) * kPkgStride;
+        float* pv = reinterpret_cast<float*>(sm + L::kPv + 512 * b);   // the package's vectors
         const uint32_t sKQ = sbase + L::kKQP + b * 32768;
 
         // ---- Gram [k;q] k^T on the tensor core; gates scan and norms meanwhile ----
@@ -854,8 +863,6 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           mma_k<8, true, 16384, true, 16384>(tmem + kColG, desc_kmajor(sKQ, 0, 16384), desc_kmajor(sKQ, 0, 16384),
                                              kIdG, false);
           mma_commit_warp(bar_pmma);
-        } else if (tid == kOutThread) {
-          finish_out();   // (before this item's vectors reuse the staging)
         }
         if (warp == 2 || warp == 3) {   // inclusive scan of g within each warp; the halves are joined below
           const int t = tid - 64, w2 = warp - 2;
@@ -904,10 +911,10 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           vCk[tid] = fast ? expf(gm - Gr) * rk : rk;
           vCw[tid] = -vB[tid] * eg * rk;
           vRho[tid] = eg * vRq[tid];
-          reinterpret_cast<float*>(sm + L::kPv)[tid] = expf(GL - Gr) * rk;
+          pv[tid] = expf(GL - Gr) * rk;
           if (tid == 0) {
-            reinterpret_cast<float*>(sm + L::kPv + 256)[0] = expf(GL);
-            reinterpret_cast<int*>(sm + L::kPv + 256)[1] = len;
+            pv[64] = expf(GL);
+            reinterpret_cast<int*>(pv)[65] = len;
           }
         }
         if (!wait_mma()) { abort = true; break; }   // (its barrier also publishes the vectors)
@@ -1055,7 +1062,9 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
               st_shared_v4(sbase + L::kN2 + sw128_off(r64, 32 * ch + 8 * c8, 0), pack8<T>(v + 8 * c8));
           }
         }
-        if (!publish(ok_s2)) { abort = true; break; }
+        // (the T stage starts overwriting the previous package's images: wait until they are read)
+        const bool ok_rd = tid != 0 || it == 0 || mbar_wait(&bar_psread[(it - 1) & 1], (uint32_t)((it - 1) >> 1) & 1u);
+        if (!publish(ok_s2 && ok_rd)) { abort = true; break; }
 
         // ---- Z = N^2 E ; T = E + Z -> T_u (shared and package), -T_w (shared) ----
         if (warp == 0) {
@@ -1144,25 +1153,10 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
               st_shared_v4(sbase + L::kA2b + sw128_off(r64, 32 * ch + 8 * c8, 0), pack8<T>(pt + 8 * c8));
           }
         }
-        // ---- the package images are complete: copy them out in bulk; the copies are
-        //      waited for during the next item, then the control warp publishes ----
+        // ---- the package images are complete: the writing warp copies them out ----
         if (!publish(ok_pw)) { abort = true; break; }
-        if (tid == kOutThread) {   // (a CTA's first package is published at once: chains are starting)
-          if (need_a1) {
-            bulk_store(pkg + kPkgA1, sm + L::kWm, 8192);
-            bulk_store(pkg + kPkgA1 + 16384, sm + L::kWm + 8192, 8192);
-            bulk_store(pkg + kPkgA1 + 8192, sm + L::kA1b, 8192);
-            bulk_store(pkg + kPkgA1 + 16384 + 8192, sm + L::kA1b + 8192, 8192);
-          }
-          bulk_store(pkg + kPkgA2, sm + L::kTu, 8192);
-          bulk_store(pkg + kPkgA2 + 8192, sm + L::kA2b, 8192);
-          bulk_store(pkg + kPkgUs, sm + L::kPv, kPkgCopy - kPkgUs);
-          bulk_commit_group();
-        }
-        out_pending = b;
-        if (it == 0 && tid == kOutThread) finish_out();
+        if (tid == 0) mbar_arrive(&bar_pstage[b]);
       }
-      if (tid == kOutThread) finish_out();
     }
   }
 

@@ -260,31 +260,30 @@ def test_a_releasing_warp_that_does_not_gate_the_buffer_can_lose_a_phase():
 
 # --------------------------------- a prep CTA's queue and its publication ---
 
-def prep_cta_run(n_chunks, P, R, K, rng, publish_when_idle=True, max_idle=20000):
+def prep_cta_run(n_chunks, P, R, K, rng, writer=True, max_idle=20000):
     """K preparing CTAs and P one-slice chains of n_chunks over a ring of R slots
     per chain. Each CTA's hand-over warp claims items into a two-entry queue
     (entry k & 1 is reused once item k - 2 is published) and waits for the
-    item's slot; its compute warps make item `it`'s package and publish it
-    while starting item it + 1 -- or at once if item it + 1 has not been handed
-    over yet (publish_when_idle), since its slot may wait for exactly that
-    package. Returns the chains' reads."""
+    item's slot; its compute warps stage item `it`'s package once the images of
+    item it - 1 have been read, and its writing warp copies each staged package
+    out and publishes it in order, on its own (writer). With writer=False the
+    package is held until the compute warps start item it + 1 (publication in
+    the next item's first stage), which can wait on the package's own slot.
+    Returns the chains' reads."""
     items = [(c, q) for c in range(n_chunks) for q in range(P)]
     nxt = [0]
     ready, consumed, slot, reads = {}, {}, {}, []
     END = object()
 
     def make_cta():
-        handed, published = {}, set()
-        pending = [None]
+        handed, staged, read, published = {}, set(), set(), set()
 
-        def publish():
-            k = pending[0]
+        def publish(k):
             c, q = handed[k]
             key = (q, c % R)
             slot[key] = c
             ready[key] = c // R + 1
             published.add(k)
-            pending[0] = None
 
         def hand_over():
             k = 0
@@ -305,19 +304,35 @@ def prep_cta_run(n_chunks, P, R, K, rng, publish_when_idle=True, max_idle=20000)
         def compute():
             it = 0
             while True:
-                if pending[0] is not None and it not in handed and publish_when_idle:
-                    publish()
                 while it not in handed:
                     yield "wait"
-                if pending[0] is not None:
-                    publish()
+                if not writer and it >= 1:
+                    read.add(it - 1)
+                    publish(it - 1)
                 if handed[it] is END:
                     return
-                pending[0] = it
+                while it >= 1 and (it - 1) not in read:
+                    yield "wait"
+                staged.add(it)
                 it += 1
                 yield "step"
 
-        return [hand_over(), compute()]
+        def write():
+            it = 0
+            while True:
+                while it not in handed:
+                    yield "wait"
+                if handed[it] is END:
+                    return
+                while it not in staged:
+                    yield "wait"
+                read.add(it)
+                yield "step"
+                publish(it)
+                it += 1
+                yield "step"
+
+        return [hand_over(), compute()] + ([write()] if writer else [])
 
     def chain(q):
         for c in range(n_chunks):
@@ -346,7 +361,7 @@ def prep_cta_run(n_chunks, P, R, K, rng, publish_when_idle=True, max_idle=20000)
 
 
 @pytest.mark.parametrize("P,R,K", [(1, 1, 1), (1, 2, 1), (2, 1, 3), (3, 2, 2), (4, 12, 6)])
-def test_prep_publishes_before_it_can_wait_on_itself(P, R, K):
+def test_prep_writer_publishes_every_package(P, R, K):
     for seed in range(20):
         reads = prep_cta_run(15, P, R, K, random.Random(seed))
         assert sorted(reads) == [(q, c) for q in range(P) for c in range(15)]
@@ -354,7 +369,7 @@ def test_prep_publishes_before_it_can_wait_on_itself(P, R, K):
 
 def test_publication_held_until_the_next_item_deadlocks_on_a_small_ring():
     with pytest.raises(AssertionError, match="deadlock"):
-        prep_cta_run(15, 1, 1, 1, random.Random(0), publish_when_idle=False)
+        prep_cta_run(15, 1, 1, 1, random.Random(0), writer=False)
 
 
 # ------------------------------ a chain CTA's MMA warp and compute warps ---
