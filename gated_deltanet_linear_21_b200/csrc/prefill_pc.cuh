@@ -172,8 +172,9 @@ struct Smem {
   static constexpr uint32_t kA1b = kWm + 16384;               // rho Q - P W [64][128], two halves 8 KB apart
   static constexpr uint32_t kA2b = kA1b + 16384;              // P T_u [64][64]
   static constexpr uint32_t kPv = kA2b + 8192;                // package vectors: us[64], gamma_L, tokens (2 x 512 B)
-  static constexpr uint32_t kAd = kPv + 1024;                 // diagonal blocks of A, fp32 [4][16][16]
-  static constexpr uint32_t kVec = kAd + 4096;                // 8 vectors of 64 fp32
+  static constexpr uint32_t kAd = kPv + 1024;                 // diagonal blocks of A, fp32 [4][16][kAdRow]
+  static constexpr int kAdRow = 20;                           // (80-byte rows: eight rows, eight bank groups)
+  static constexpr uint32_t kVec = kAd + 4 * 16 * kAdRow * 4; // 8 vectors of 64 fp32
   static constexpr uint32_t kQueue = kVec + 8 * 256;          // 2 items handed over by the control warp:
   static constexpr uint32_t kQueueBytes = 640;                //   {valid, s, q, len}, g[64] @64, beta[64] @320
   static constexpr uint32_t kRounds = kQueue + 2 * kQueueBytes;      // round_start[kMaxRounds + 1]
@@ -952,13 +953,15 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             }
             const int blk = rr >> 4;
             if ((blk >> 1) == ch) {
-              float* dst = Ad + (blk * 16 + (rr & 15)) * 16;
-              if (blk & 1) {
+              float4* dst = reinterpret_cast<float4*>(Ad + (blk * 16 + (rr & 15)) * L::kAdRow);
+              if (blk & 1) {   // (constant indices keep x in registers)
 #pragma unroll
-                for (int q2 = 0; q2 < 16; ++q2) dst[q2] = x[16 + q2];
+                for (int q4 = 0; q4 < 4; ++q4)
+                  dst[q4] = make_float4(x[16 + 4 * q4], x[17 + 4 * q4], x[18 + 4 * q4], x[19 + 4 * q4]);
               } else {
 #pragma unroll
-                for (int q2 = 0; q2 < 16; ++q2) dst[q2] = x[q2];
+                for (int q4 = 0; q4 < 4; ++q4)
+                  dst[q4] = make_float4(x[4 * q4], x[1 + 4 * q4], x[2 + 4 * q4], x[3 + 4 * q4]);
               }
             }
 #pragma unroll
@@ -991,17 +994,17 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         // ---- D = (I + A_d)^-1 ----
         if (tid < 64) {
           const int blk = tid >> 4, jj = tid & 15;
-          const float* Ab = Ad + blk * 256;
+          const float* Ab = Ad + blk * 16 * L::kAdRow;
           float xs[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             float acc0 = 0.f, acc1 = 0.f;   // two chains halve the dependent FMA latency
 #pragma unroll
             for (int k2 = 0; k2 + 1 < i; k2 += 2) {
-              acc0 = fmaf(Ab[i * 16 + k2], xs[k2], acc0);
-              acc1 = fmaf(Ab[i * 16 + k2 + 1], xs[k2 + 1], acc1);
+              acc0 = fmaf(Ab[i * L::kAdRow + k2], xs[k2], acc0);
+              acc1 = fmaf(Ab[i * L::kAdRow + k2 + 1], xs[k2 + 1], acc1);
             }
-            if (i & 1) acc0 = fmaf(Ab[i * 16 + i - 1], xs[i - 1], acc0);
+            if (i & 1) acc0 = fmaf(Ab[i * L::kAdRow + i - 1], xs[i - 1], acc0);
             xs[i] = (i == jj) ? 1.f : (i > jj ? -(acc0 + acc1) : 0.f);
           }
 #pragma unroll
