@@ -878,23 +878,27 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           if (lane == 0) scan[2 + w2] = nonpos == 0xffffffffu ? 1.f : 0.f;
           vB[t] = reinterpret_cast<const float*>(qe + 80)[t];
           vG[t] = gv;
-        } else if (warp >= 4) {   // norms, one row each: rows 0-63 k, rows 64-127 q
-          const int row = tid - 128;
-          float ss0 = 0.f, ss1 = 0.f;
+        }
+        {   // squared norms of the [k;q] rows in halves, two threads a row (rows 0-63 k, 64-127 q):
+            // warps 0-3 columns 0-63, warps 4-7 columns 64-127, four accumulators a thread. The
+            // partial sums go to vCk/vCw (half 0) and vRho/vGf (half 1), which the thread of the
+            // vector step below reads before it writes those same four entries.
+          const int row = tid & 127, half = tid >> 7;
+          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-          for (int c8 = 0; c8 < 16; ++c8) {
+          for (int c8 = 0; c8 < 8; ++c8) {
             float f[8];
-            unpack8<T>(ld_shared_v4(sKQ + sw128_off(row, 8 * c8, 16384)), f);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              if (e & 1) ss1 = fmaf(f[2 * e], f[2 * e], fmaf(f[2 * e + 1], f[2 * e + 1], ss1));
-              else ss0 = fmaf(f[2 * e], f[2 * e], fmaf(f[2 * e + 1], f[2 * e + 1], ss0));
-            }
+            unpack8<T>(ld_shared_v4(sKQ + sw128_off(row, 64 * half + 8 * c8, 16384)), f);
+            a0 = fmaf(f[0], f[0], a0);
+            a1 = fmaf(f[1], f[1], a1);
+            a2 = fmaf(f[2], f[2], a2);
+            a3 = fmaf(f[3], f[3], a3);
+            a0 = fmaf(f[4], f[4], a0);
+            a1 = fmaf(f[5], f[5], a1);
+            a2 = fmaf(f[6], f[6], a2);
+            a3 = fmaf(f[7], f[7], a3);
           }
-          const float ss = ss0 + ss1;
-          const int rr = row & 63;
-          if (row < 64) vRk[rr] = rr < len ? 1.0f / sqrtf(ss + kNormEps) : 0.f;
-          else vRq[rr] = rr < len ? p.scale / sqrtf(ss + kNormEps) : 0.f;
+          (half ? vRho : vCk)[row] = (a0 + a1) + (a2 + a3);   // (vCw, vGf follow vCk, vRho)
         }
         cbar();
 
@@ -906,12 +910,16 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         const float gm = 0.5f * (G0 + GL);
         if (tid < 64) {
           const float Gr = vG[tid] + (tid >= 32 ? s0 : 0.f);
-          const float rk = vRk[tid];
+          const float ssk = vCk[tid] + vRho[tid], ssq = vCw[tid] + vGf[tid];
+          const float rk = tid < len ? 1.0f / sqrtf(ssk + kNormEps) : 0.f;
+          const float rq = tid < len ? p.scale / sqrtf(ssq + kNormEps) : 0.f;
+          vRk[tid] = rk;
+          vRq[tid] = rq;
           const float eg = expf(Gr);
           vGf[tid] = Gr;
           vCk[tid] = fast ? expf(gm - Gr) * rk : rk;
           vCw[tid] = -vB[tid] * eg * rk;
-          vRho[tid] = eg * vRq[tid];
+          vRho[tid] = eg * rq;
           pv[tid] = expf(GL - Gr) * rk;
           if (tid == 0) {
             pv[64] = expf(GL);
