@@ -627,6 +627,34 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     }
   } else {
     // ============================== prep role ===============================
+    // The hand-over warp first prefetches into L2 the raw tiles and gates of the CTA's
+    // first item (fixed: items [0, prep CTAs) go one to each) as it lies in round 0,
+    // where it is chunk c of chain q with item = c P0 + q (P0 the round's chains), so
+    // that the hand-over's loads find them there; a guess outside the chain's
+    // chunks prefetches nothing.
+    if (is_ctl) {
+      const long p0 = min((long)chains_per_round, n_chains);
+      const long item = (long)blockIdx.x - NC;
+      if (p0 > 0 && item >= 0) {
+        const long j = item % p0;
+        int tb, te;
+        seq_bounds((int)(j / Hv), tb, te);
+        const int c0 = tb + (int)(item / p0) * kC;
+        if (c0 < te) {
+          const int h = (int)(j % Hv), hq = h / (Hv / Hqk);
+          if (lane == 0) {
+            tma_prefetch_3d(&kmap, 0, hq, c0);
+            tma_prefetch_3d(&kmap, 64, hq, c0);
+            tma_prefetch_3d(&qmap, 0, hq, c0);
+            tma_prefetch_3d(&qmap, 64, hq, c0);
+          }
+          for (int e = lane; e < kC && c0 + e < te; e += 32) {
+            prefetch_l2(p.g + (size_t)(c0 + e) * Hv + h);
+            prefetch_l2(p.beta + (size_t)(c0 + e) * Hv + h);
+          }
+        }
+      }
+    }
     // round table: items of round r are [round_start[r], round_start[r+1])
     const int n_rounds = (int)min((n_slice_chains + NC - 1) / NC, (long)kMaxRounds);
     // the longest chain of each round (warps over rounds, lanes over its chains) ...
