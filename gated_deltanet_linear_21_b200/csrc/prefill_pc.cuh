@@ -439,6 +439,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           for (int kk = 0; kk < 8; ++kk)
             tmem_cp_128x256b_warp(tmem + kColA1 + 64u * ab + 8u * kk, desc_advance(a0, kmajor_step(kk, 16384)));
         };
+        const uint64_t s0 = desc_mnmajor(sSb, 0, kRB, 128 * kRB);   // S^T, the B operand of A1 S^T
         long gc = 0;
         bool early = false;
         uint32_t ph_u = 0, ph_s = 0;
@@ -451,15 +452,15 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             const int b = (int)(gc % NB);
             const uint32_t in = sbase + L::kIn + b * L::kInBytes;
             const uint32_t ycol = kColY + 128u * (uint32_t)(gc & 1);   // two Y buffers in TMEM
+            const uint32_t ab = (uint32_t)(gc & 1);                     // the A1 buffer in TMEM
+            // (a first chunk from a zero state has no A1 S^T; its package carries no A1)
+            const bool a1s = c > 0 || p.state_in != nullptr;
             if (!mbar_wait(&bar_full[b], (uint32_t)(gc / NB) & 1u) || !mbar_wait(bar_s, ph_s)) { abort = true; break; }
             ph_s ^= 1;
             __syncwarp();
             tc_fence_after();
-            const uint32_t ab = (uint32_t)(gc & 1);   // the A1 buffer in TMEM
             if (!early) issue_a2v(b, ycol);
-            if (c > 0 || p.state_in != nullptr) {   // (a first chunk from a zero state has no A1 S^T;
-                                                    //  its package carries no A1)
-              const uint64_t s0 = desc_mnmajor(sSb, 0, kRB, 128 * kRB);
+            if (a1s) {
               if (early) {   // A1 was staged in TMEM while the previous chunk ran
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
