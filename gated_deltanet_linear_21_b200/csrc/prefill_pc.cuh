@@ -440,6 +440,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             tmem_cp_128x256b_warp(tmem + kColA1 + 64u * ab + 8u * kk, desc_advance(a0, kmajor_step(kk, 16384)));
         };
         const uint64_t s0 = desc_mnmajor(sSb, 0, kRB, 128 * kRB);   // S^T, the B operand of A1 S^T
+        const uint64_t u0 = desc_mnmajor(sUsb, 0, kRB, 64 * kRB);   // U_s, the B operand of dS
         long gc = 0;
         bool early = false;
         uint32_t ph_u = 0, ph_s = 0;
@@ -471,12 +472,12 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
               }
             }
             mma_commit_warp(bar_mma);
+            const uint64_t kd = desc_mnmajor(in + L::kInK, 0, 128, 8192);   // K_raw^T, the A operand of dS
             if (!mbar_wait(bar_u, ph_u)) { abort = true; break; }
             ph_u ^= 1;
             __syncwarp();
             tc_fence_after();
-            mma_k<4, false, 128, false, kRB>(tmem + kColDS, desc_mnmajor(in + L::kInK, 0, 128, 8192),
-                                             desc_mnmajor(sUsb, 0, kRB, 64 * kRB), kIdDS, false);
+            mma_k<4, false, 128, false, kRB>(tmem + kColDS, kd, u0, kIdDS, false);
             mma_commit_warp(bar_ds);
             // the other Y buffer was last read in chunk gc - 1, whose epilogues all ended
             // before the compute warps' state update of that chunk (and so before bar_u);
