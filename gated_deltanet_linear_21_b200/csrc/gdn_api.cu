@@ -244,8 +244,8 @@ struct PcPlan {
   long nc;
 };
 PcPlan plan_pc(long chains, int64_t total_T, int n_seqs, int Hv, int sms) {
-  const double kChainStep[3] = {2200.0, 2600.0, 3400.0};   // DVP 32, 64, 128
-  const double kPrepItem = 10300.0;
+  const double kChainStep[3] = {1950.0, 2300.0, 3100.0};   // DVP 32, 64, 128
+  const double kPrepItem = 10500.0;
   const double chunks = std::max(1.0, std::ceil((double)total_T / std::max(1, n_seqs) / 64.0));
   PcPlan best = {128, 1};
   double best_t = 1e300;
