@@ -183,7 +183,7 @@ struct Smem {
   // common
   static constexpr uint32_t kCommon = ((kChainEnd > kPrepEnd ? kChainEnd : kPrepEnd) + 7) & ~7u;
   static constexpr uint32_t kBarA = kCommon;                  // mbarriers (chain 9, prep 16)
-  static constexpr uint32_t kMisc = kBarA + 16 * 8;           // tmem slot, scan[4]
+  static constexpr uint32_t kMisc = kBarA + 16 * 8;           // tmem slot
   static constexpr uint32_t kTotal = kMisc + 64;
   static constexpr uint32_t kAlloc = kTotal + 1024;
   static_assert(kAlloc <= 227 * 1024, "shared memory budget");
@@ -259,7 +259,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
   uint64_t* bar_ds = bar_mma + 2;          // the dS product's commits
   uint64_t* bar_s = bar_mma + 3;           // the 16-bit state copy is written (the 8 compute warps)
   uint64_t* bar_o = bar_mma + 4;           // O staged for the TMA store (the 4 O warps)
-  uint32_t* misc = reinterpret_cast<uint32_t*>(sm + L::kMisc);     // [0] tmem, [2..5] scan
+  uint32_t* misc = reinterpret_cast<uint32_t*>(sm + L::kMisc);     // [0] tmem
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qd = warp & 3, ch = (warp >> 2) & 1;
@@ -380,8 +380,9 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           const int c0 = t_begin + c * kC;
           mbar_arrive_expect_tx_warp(&bar_full[b], kPkgCopy + 16384 + 64 * kR);
           bulk_load_warp(dst, ring + (size_t)slot * kPkgStride, kPkgCopy, &bar_full[b]);
-          tma_load_3d_warp(dst + L::kInK, &kmap, &bar_full[b], 0, hq, c0);
-          tma_load_3d_warp(dst + L::kInK + 8192, &kmap, &bar_full[b], 64, hq, c0);
+          // (the chains' k reads are its last: the prep CTAs read it before the package exists)
+          tma_load_3d_warp_hint(dst + L::kInK, &kmap, &bar_full[b], 0, hq, c0, l2_evict_first_policy());
+          tma_load_3d_warp_hint(dst + L::kInK + 8192, &kmap, &bar_full[b], 64, hq, c0, l2_evict_first_policy());
 #pragma unroll
           for (int vb = 0; vb < L::kBlocks; ++vb)
             tma_load_3d_warp_hint(dst + L::kInV + vb * 64 * L::kRB, &vmap, &bar_full[b], i0 + vb * L::kBlk, h, c0,
@@ -417,6 +418,10 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       }
     } else if (warp == kMmaWarp || warp < 8) {
       constexpr uint32_t kIdY = idesc_f16kind(128, DVP, false, true, kFmt);
+      // Each group of the chain's K-steps from one asm block (mma_run_warp) at 32-row slices,
+      // one block a step at wider ones: measured side by side on the B200, either way round
+      // costs 0.5-1 % of the call.
+      constexpr bool kBatchedIssue = DVP == 32;
       constexpr uint32_t kIdDS = idesc_f16kind(128, DVP, true, true, kFmt);
       const uint32_t sSb = sbase + L::kSb;
       const uint32_t sUsb = sbase + L::kUsb;
@@ -428,8 +433,11 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         //      warps through mbarriers (bounded) ----
         auto issue_a2v = [&](int b, uint32_t ycol) {   // A2 V_raw of input buffer b, the first term of Y
           const uint32_t in = sbase + L::kIn + b * L::kInBytes;
-          mma_k<4, true, 0, false, kRB>(tmem + ycol, desc_kmajor(in + kPkgA2, 0, 0),
-                                        desc_mnmajor(in + L::kInV, 0, kRB, 64 * kRB), kIdY, false);
+          const uint64_t a2 = desc_kmajor(in + kPkgA2, 0, 0), v0 = desc_mnmajor(in + L::kInV, 0, kRB, 64 * kRB);
+          if constexpr (kBatchedIssue)
+            mma_run_warp<4, 2, kRB>(tmem + ycol, a2, v0, kIdY, 0u);
+          else
+            mma_k<4, true, 0, false, kRB>(tmem + ycol, a2, v0, kIdY, false);
         };
         // the package's A1 (input buffer b) into TMEM buffer ab, so that A1 S^T reads
         // only S^T from shared memory on the chain (the copy is ordered before it)
@@ -463,10 +471,14 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             if (!early) issue_a2v(b, ycol);
             if (a1s) {
               if (early) {   // A1 was staged in TMEM while the previous chunk ran
+                if constexpr (kBatchedIssue) {
+                  mma8_tmem_a_run_warp<kRB>(tmem + ycol, tmem + kColA1 + 64u * ab, s0, kIdY);
+                } else {
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                  mma_f16_tmem_a_warp(tmem + ycol, tmem + kColA1 + 64u * ab + 8u * kk,
-                                      desc_advance(s0, mnmajor_step(kk, kRB)), kIdY, 1u);
+                  for (int kk = 0; kk < 8; ++kk)
+                    mma_f16_tmem_a_warp(tmem + ycol, tmem + kColA1 + 64u * ab + 8u * kk,
+                                        desc_advance(s0, mnmajor_step(kk, kRB)), kIdY, 1u);
+                }
               } else {       // staging it now would only add a pass: read it from shared memory
                 mma_k<8, true, 16384, false, kRB>(tmem + ycol, desc_kmajor(in + kPkgA1, 0, 16384), s0, kIdY, true);
               }
@@ -477,7 +489,10 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             ph_u ^= 1;
             __syncwarp();
             tc_fence_after();
-            mma_k<4, false, 128, false, kRB>(tmem + kColDS, kd, u0, kIdDS, false);
+            if constexpr (kBatchedIssue)
+              mma_run_warp<4, 128, kRB>(tmem + kColDS, kd, u0, kIdDS, 0u);
+            else
+              mma_k<4, false, 128, false, kRB>(tmem + kColDS, kd, u0, kIdDS, false);
             mma_commit_warp(bar_ds);
             // the other Y buffer was last read in chunk gc - 1, whose epilogues all ended
             // before the compute warps' state update of that chunk (and so before bar_u);
@@ -784,8 +799,9 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           mbar_expect_tx_warp(&bar_pfull[b], 4 * 8192);
           tma_load_3d_warp(kq, &kmap, &bar_pfull[b], 0, hq, c0);
           tma_load_3d_warp(kq + 16384, &kmap, &bar_pfull[b], 64, hq, c0);
-          tma_load_3d_warp(kq + 8192, &qmap, &bar_pfull[b], 0, hq, c0);
-          tma_load_3d_warp(kq + 16384 + 8192, &qmap, &bar_pfull[b], 64, hq, c0);
+          // (q's only readers are the prep items of the group's v heads, handed out together)
+          tma_load_3d_warp_hint(kq + 8192, &qmap, &bar_pfull[b], 0, hq, c0, l2_evict_first_policy());
+          tma_load_3d_warp_hint(kq + 16384 + 8192, &qmap, &bar_pfull[b], 64, hq, c0, l2_evict_first_policy());
           float* qg = reinterpret_cast<float*>(qe + 16);
           float* qb = reinterpret_cast<float*>(qe + 80);
 #pragma unroll
@@ -858,8 +874,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       // ---- compute warps ----
       constexpr uint32_t kIdG = idesc_f16kind(128, 64, false, false, kFmt);
       constexpr uint32_t kId64 = idesc_f16kind(64, 64, false, true, kFmt);
-      float* vG = reinterpret_cast<float*>(sm + L::kVec);   // per-warp partial scan of g
-      float* vB = vG + 64;
+      float* vB = reinterpret_cast<float*>(sm + L::kVec) + 64;   // beta (after 64 spare floats)
       float* vRk = vB + 64;
       float* vRq = vRk + 64;
       float* vCk = vRq + 64;
@@ -867,7 +882,6 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       float* vRho = vCw + 64;
       float* vGf = vRho + 64;                               // G_r
       float* Ad = reinterpret_cast<float*>(sm + L::kAd);
-      float* scan = reinterpret_cast<float*>(&misc[2]);
 
       for (int it = 0; !abort; ++it) {
         const int b = it & 1;
@@ -889,36 +903,40 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         float* pv = reinterpret_cast<float*>(sm + L::kPv + 512 * b);   // the package's vectors
         const uint32_t sKQ = sbase + L::kKQP + b * 32768;
 
-        // ---- Gram [k;q] k^T on the tensor core; gates scan and norms meanwhile ----
+        // ---- Gram [k;q] k^T on the tensor core; meanwhile the gates' scan, the norms and the row scales ----
         if (warp == 0) {
-          mma_k<8, true, 16384, true, 16384>(tmem + kColG, desc_kmajor(sKQ, 0, 16384), desc_kmajor(sKQ, 0, 16384),
-                                             kIdG, false);
+          const uint64_t g0 = desc_kmajor(sKQ, 0, 16384);   // (K 64-127 in the tile's second 16 KB)
+          mma_run_warp<4, 2, 2>(tmem + kColG, g0, g0, kIdG, 0u);
+          mma_run_warp<4, 2, 2>(tmem + kColG, desc_advance(g0, 16384), desc_advance(g0, 16384), kIdG, 1u);
           mma_commit_warp(bar_pmma);
         }
-        if (warp == 2 || warp == 3) {   // inclusive scan of g within each warp; the halves are joined below
-          const int t = tid - 64, w2 = warp - 2;
-          float gv = reinterpret_cast<const float*>(qe + 16)[t];
-          const unsigned nonpos = __ballot_sync(0xffffffffu, gv <= 0.f);
+        // every warp scans the chunk's gates itself (two values a lane): G_r for rows lane, 32 + lane
+        const float* qg = reinterpret_cast<const float*>(qe + 16);
+        float g0 = qg[lane], g1 = qg[32 + lane];
+        const bool nonpos = __all_sync(0xffffffffu, g0 <= 0.f && g1 <= 0.f);
 #pragma unroll
-          for (int off = 1; off < 32; off <<= 1) {
-            const float up = __shfl_up_sync(0xffffffffu, gv, off);
-            if (lane >= off) gv += up;
+        for (int off = 1; off < 32; off <<= 1) {
+          const float u0 = __shfl_up_sync(0xffffffffu, g0, off);
+          const float u1 = __shfl_up_sync(0xffffffffu, g1, off);
+          if (lane >= off) {
+            g0 += u0;
+            g1 += u1;
           }
-          if (lane == 31) scan[w2] = gv;
-          if (lane == 0) scan[2 + w2] = nonpos == 0xffffffffu ? 1.f : 0.f;
-          vB[t] = reinterpret_cast<const float*>(qe + 80)[t];
-          vG[t] = gv;
         }
-        {   // squared norms of the [k;q] rows in halves, two threads a row (rows 0-63 k, 64-127 q):
-            // warps 0-3 columns 0-63, warps 4-7 columns 64-127, four accumulators a thread. The
-            // partial sums go to vCk/vCw (half 0) and vRho/vGf (half 1), which the thread of the
-            // vector step below reads before it writes those same four entries.
-          const int row = tid & 127, half = tid >> 7;
+        const float s0 = __shfl_sync(0xffffffffu, g0, 31);
+        g1 += s0;
+        const float G0 = __shfl_sync(0xffffffffu, g0, 0);
+        const float GL = __shfl_sync(0xffffffffu, len - 1 < 32 ? g0 : g1, (len - 1) & 31);
+        const bool fast = nonpos && (G0 - GL) <= 160.f;
+        const float gm = 0.5f * (G0 + GL);
+        {   // squared norm of row 16 warp + lane / 2 of [k;q] (warps 0-3 k rows, 4-7 q rows) in two
+            // halves on adjacent lanes, four accumulators a lane; then that row's scales
+          const int nrow = 16 * warp + (lane >> 1), nhalf = lane & 1;
           float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
           for (int c8 = 0; c8 < 8; ++c8) {
             float f[8];
-            unpack8<T>(ld_shared_v4(sKQ + sw128_off(row, 64 * half + 8 * c8, 16384)), f);
+            unpack8<T>(ld_shared_v4(sKQ + sw128_off(nrow, 64 * nhalf + 8 * c8, 16384)), f);
             a0 = fmaf(f[0], f[0], a0);
             a1 = fmaf(f[1], f[1], a1);
             a2 = fmaf(f[2], f[2], a2);
@@ -928,29 +946,30 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             a2 = fmaf(f[6], f[6], a2);
             a3 = fmaf(f[7], f[7], a3);
           }
-          (half ? vRho : vCk)[row] = (a0 + a1) + (a2 + a3);   // (vCw, vGf follow vCk, vRho)
-        }
-        cbar();
-
-        // ---- decay vectors; the package's row scales ----
-        const float s0 = scan[0];
-        const float G0 = vG[0];
-        const float GL = vG[len - 1] + (len - 1 >= 32 ? s0 : 0.f);
-        const bool fast = scan[2] > 0.f && scan[3] > 0.f && (G0 - GL) <= 160.f;
-        const float gm = 0.5f * (G0 + GL);
-        if (tid < 64) {
-          const float Gr = vG[tid] + (tid >= 32 ? s0 : 0.f);
-          const float ssk = vCk[tid] + vRho[tid], ssq = vCw[tid] + vGf[tid];
-          const float rk = tid < len ? 1.0f / sqrtf(ssk + kNormEps) : 0.f;
-          const float rq = tid < len ? p.scale / sqrtf(ssq + kNormEps) : 0.f;
-          vRk[tid] = rk;
-          vRq[tid] = rq;
+          const float part = (a0 + a1) + (a2 + a3);
+          const float other = __shfl_xor_sync(0xffffffffu, part, 1);
+          const float ss = nhalf ? other + part : part + other;   // (the first half's sum first)
+          const int r = nrow & 63;
+          const float Ga = __shfl_sync(0xffffffffu, g0, r & 31), Gb = __shfl_sync(0xffffffffu, g1, r & 31);
+          const float Gr = r < 32 ? Ga : Gb;
           const float eg = expf(Gr);
-          vGf[tid] = Gr;
-          vCk[tid] = fast ? expf(gm - Gr) * rk : rk;
-          vCw[tid] = -vB[tid] * eg * rk;
-          vRho[tid] = eg * rq;
-          pv[tid] = expf(GL - Gr) * rk;
+          if (warp < 4) {
+            const float rk = r < len ? 1.0f / sqrtf(ss + kNormEps) : 0.f;
+            if (nhalf == 0) {
+              vRk[r] = rk;
+              vCk[r] = fast ? expf(gm - Gr) * rk : rk;
+              pv[r] = expf(GL - Gr) * rk;
+            } else {
+              const float bt = reinterpret_cast<const float*>(qe + 80)[r];
+              vB[r] = bt;
+              vGf[r] = Gr;
+              vCw[r] = -bt * eg * rk;
+            }
+          } else if (nhalf == 0) {
+            const float rq = r < len ? p.scale / sqrtf(ss + kNormEps) : 0.f;
+            vRq[r] = rq;
+            vRho[r] = eg * rq;
+          }
           if (tid == 0) {
             pv[64] = expf(GL);
             reinterpret_cast<int*>(pv)[65] = len;
@@ -1059,8 +1078,8 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
 
         // ---- N = D A_o ----
         if (warp == 0) {
-          mma_k<4, true, 0, false, 128>(tmem + kColN, desc_kmajor(sbase + L::kDm, 0, 0),
-                                        desc_mnmajor(sbase + L::kAo, 0, 128, 8192), kId64, false);
+          mma_run_warp<4, 2, 128>(tmem + kColN, desc_kmajor(sbase + L::kDm, 0, 0),
+                                        desc_mnmajor(sbase + L::kAo, 0, 128, 8192), kId64, 0u);
           mma_commit_warp(bar_pmma);
         }
         const bool ok_n = wait_mma_local();
@@ -1078,11 +1097,14 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         // ---- N D (lanes 0-15) and N^2 (lanes 16-31) ----
         if (warp == 0) {
           const uint64_t nm = desc_kmajor(sbase + L::kNm, 0, 0);
-          mma_k<4, true, 0, false, 128>(tmem + kColS2, nm, desc_mnmajor(sbase + L::kDm, 0, 128, 8192), kId64, false);
-          mma_k<4, true, 0, false, 128>(tmem + (16u << 16) + kColS2, nm, desc_mnmajor(sbase + L::kNm, 0, 128, 8192),
-                                        kId64, false);
+          mma_run_warp<4, 2, 128>(tmem + kColS2, nm, desc_mnmajor(sbase + L::kDm, 0, 128, 8192), kId64, 0u);
+          mma_run_warp<4, 2, 128>(tmem + (16u << 16) + kColS2, nm, desc_mnmajor(sbase + L::kNm, 0, 128, 8192),
+                                        kId64, 0u);
           mma_commit_warp(bar_pmma);
         }
+        uint4 dq[4];   // (D is final since its stage: read before the wait)
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8) dq[c8] = ld_shared_v4(sbase + L::kDm + sw128_off(r64, 32 * ch + 8 * c8, 0));
         const bool ok_s2 = wait_mma_local();
         float E[32];   // lanes 0-15: columns 32ch..32ch+31 of row r64 of E = D - N D (fp32)
         {
@@ -1092,7 +1114,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
 #pragma unroll
             for (int c8 = 0; c8 < 4; ++c8) {
               float df[8];
-              unpack8<T>(ld_shared_v4(sbase + L::kDm + sw128_off(r64, 32 * ch + 8 * c8, 0)), df);
+              unpack8<T>(dq[c8], df);
 #pragma unroll
               for (int e = 0; e < 8; ++e) E[8 * c8 + e] = df[e] - v[8 * c8 + e];
               st_shared_v4(sbase + L::kEm + sw128_off(r64, 32 * ch + 8 * c8, 0), pack8<T>(E + 8 * c8));
@@ -1109,8 +1131,8 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
 
         // ---- Z = N^2 E ; T = E + Z -> T_u (shared and package), -T_w (shared) ----
         if (warp == 0) {
-          mma_k<4, true, 0, false, 128>(tmem + kColZ, desc_kmajor(sbase + L::kN2, 0, 0),
-                                        desc_mnmajor(sbase + L::kEm, 0, 128, 8192), kId64, false);
+          mma_run_warp<4, 2, 128>(tmem + kColZ, desc_kmajor(sbase + L::kN2, 0, 0),
+                                        desc_mnmajor(sbase + L::kEm, 0, 128, 8192), kId64, 0u);
           mma_commit_warp(bar_pmma);
         }
         const bool ok_z = wait_mma_local();
@@ -1120,13 +1142,21 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           if (lo16) {
 #pragma unroll
             for (int c8 = 0; c8 < 4; ++c8) {
-              float tu[8], tw[8];
+              float tu[8], tw[8], bb[8], ww[8];
+              {
+                const float4* b4 = reinterpret_cast<const float4*>(vB + 32 * ch + 8 * c8);
+                const float4* w4 = reinterpret_cast<const float4*>(vCw + 32 * ch + 8 * c8);
+                const float4 b0 = b4[0], b1 = b4[1], w0 = w4[0], w1 = w4[1];
+                bb[0] = b0.x; bb[1] = b0.y; bb[2] = b0.z; bb[3] = b0.w;
+                bb[4] = b1.x; bb[5] = b1.y; bb[6] = b1.z; bb[7] = b1.w;
+                ww[0] = w0.x; ww[1] = w0.y; ww[2] = w0.z; ww[3] = w0.w;
+                ww[4] = w1.x; ww[5] = w1.y; ww[6] = w1.z; ww[7] = w1.w;
+              }
 #pragma unroll
               for (int e = 0; e < 8; ++e) {
-                const int sidx = 32 * ch + 8 * c8 + e;
                 const float t = E[8 * c8 + e] + z[8 * c8 + e];
-                tu[e] = t * vB[sidx];
-                tw[e] = t * vCw[sidx];
+                tu[e] = t * bb[e];
+                tw[e] = t * ww[e];
               }
               const uint32_t off = sw128_off(r64, 32 * ch + 8 * c8, 0);
               st_shared_v4(sbase + L::kTu + off, pack8<T>(tu));
@@ -1142,9 +1172,9 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         if (need_a1) {
           if (warp == 0) {
             const uint64_t tw = desc_kmajor(sbase + L::kTw, 0, 0);
-            mma_k<4, true, 0, false, 128>(tmem + kColW, tw, desc_mnmajor(sKQ, 0, 128, 16384), kId64, false);
-            mma_k<4, true, 0, false, 128>(tmem + (16u << 16) + kColW, tw, desc_mnmajor(sKQ + 16384, 0, 128, 16384),
-                                          kId64, false);
+            mma_run_warp<4, 2, 128>(tmem + kColW, tw, desc_mnmajor(sKQ, 0, 128, 16384), kId64, 0u);
+            mma_run_warp<4, 2, 128>(tmem + (16u << 16) + kColW, tw, desc_mnmajor(sKQ + 16384, 0, 128, 16384),
+                                          kId64, 0u);
             mma_commit_warp(bar_pmma);
           }
           const bool ok_w = wait_mma_local();
@@ -1161,18 +1191,21 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         // ---- -P W and P T_u -> A1 rows 64-127 = rho Q_raw - P W, A2 rows 64-127 = P T_u ----
         if (warp == 0) {
           if (need_a1) {
-            mma_k<4, true, 0, false, 128>(tmem + kColPW, desc_kmajor(sbase + L::kPm, 0, 0),
-                                          desc_mnmajor(sbase + L::kWm, 0, 128, 8192), kId64, false);
-            mma_k<4, true, 0, false, 128>(tmem + (16u << 16) + kColPW, desc_kmajor(sbase + L::kPm, 0, 0),
-                                          desc_mnmajor(sbase + L::kWm + 8192, 0, 128, 8192), kId64, false);
+            mma_run_warp<4, 2, 128>(tmem + kColPW, desc_kmajor(sbase + L::kPm, 0, 0),
+                                          desc_mnmajor(sbase + L::kWm, 0, 128, 8192), kId64, 0u);
+            mma_run_warp<4, 2, 128>(tmem + (16u << 16) + kColPW, desc_kmajor(sbase + L::kPm, 0, 0),
+                                          desc_mnmajor(sbase + L::kWm + 8192, 0, 128, 8192), kId64, 0u);
           }
-          mma_k<4, true, 0, false, 128>(tmem + kColPT, desc_kmajor(sbase + L::kPm, 0, 0),
-                                        desc_mnmajor(sbase + L::kTu, 0, 128, 8192), kId64, false);
+          mma_run_warp<4, 2, 128>(tmem + kColPT, desc_kmajor(sbase + L::kPm, 0, 0),
+                                        desc_mnmajor(sbase + L::kTu, 0, 128, 8192), kId64, 0u);
           mma_commit_warp(bar_pmma);
         }
+        uint4 qq[4];   // (the raw q tile and rho are final: read before the wait)
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8) qq[c8] = ld_shared_v4(sKQ + sw128_off(64 + r64, dhalf + 8 * c8, 16384));
+        const float rho = vRho[r64];
         const bool ok_pw = wait_mma_local();
         {
-          const float rho = vRho[r64];
           if (need_a1) {
             float pw[32];
             tmem_ld32(tmem + tlane + kColPW + 32 * ch, pw);
@@ -1180,7 +1213,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             for (int c8 = 0; c8 < 4; ++c8) {
               const int d = dhalf + 8 * c8;
               float qf[8], a[8];
-              unpack8<T>(ld_shared_v4(sKQ + sw128_off(64 + r64, d, 16384)), qf);
+              unpack8<T>(qq[c8], qf);
 #pragma unroll
               for (int e = 0; e < 8; ++e) a[e] = fmaf(rho, qf[e], pw[8 * c8 + e]);
               st_shared_v4(sbase + L::kA1b + sw128_off(r64, d, 8192), pack8<T>(a));

@@ -424,6 +424,59 @@ __device__ __forceinline__ void mma_k(uint32_t d_tmem, uint64_t a0, uint64_t b0,
   }
 }
 
+// The same as mma_k for NK = 4 or 8 steps whose descriptors advance by the same
+// ASTEP / BSTEP 16-byte units every step, from one asm block: one elect.sync and
+// the steps' address arithmetic as immediates, so that the elected lane issues the
+// whole group back to back. acc as in mma_k (the first step; the others accumulate).
+#define GDN_MMA_NEXT                                                       \
+  "add.s64 a, a, %5;\n\t"                                                  \
+  "add.s64 b, b, %6;\n\t"                                                  \
+  "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t"
+#define GDN_MMA_HEAD                                                       \
+  "{\n\t.reg .pred e, p, t;\n\t.reg .b64 a, b;\n\t"                        \
+  "setp.ne.b32 p, %4, 0;\n\t"                                              \
+  "setp.eq.b32 t, %4, %4;\n\t"                                             \
+  "mov.b64 a, %1;\n\t"                                                     \
+  "mov.b64 b, %2;\n\t"                                                     \
+  "elect.sync _|e, 0xffffffff;\n\t"                                        \
+  "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, p;\n\t"
+template <int NK, uint32_t ASTEP, uint32_t BSTEP>
+__device__ __forceinline__ void mma_run_warp(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint32_t idesc, uint32_t acc) {
+  static_assert(NK == 4 || NK == 8, "4 or 8 steps");
+  if constexpr (NK == 4) {
+    asm volatile(GDN_MMA_HEAD GDN_MMA_NEXT GDN_MMA_NEXT GDN_MMA_NEXT "}" ::"r"(d_tmem), "l"(a0), "l"(b0),
+                 "r"(idesc), "r"(acc), "n"(ASTEP), "n"(BSTEP)
+                 : "memory");
+  } else {
+    asm volatile(GDN_MMA_HEAD GDN_MMA_NEXT GDN_MMA_NEXT GDN_MMA_NEXT GDN_MMA_NEXT GDN_MMA_NEXT GDN_MMA_NEXT
+                     GDN_MMA_NEXT "}" ::"r"(d_tmem),
+                 "l"(a0), "l"(b0), "r"(idesc), "r"(acc), "n"(ASTEP), "n"(BSTEP)
+                 : "memory");
+  }
+}
+#undef GDN_MMA_HEAD
+#undef GDN_MMA_NEXT
+// Eight accumulating K-steps with A in TMEM (8 columns a step from a_tmem) and B
+// advancing BSTEP 16-byte units a step, from one asm block (as mma_run_warp).
+#define GDN_MMA_TA_NEXT                                                    \
+  "add.u32 a, a, 8;\n\t"                                                   \
+  "add.s64 b, b, %4;\n\t"                                                  \
+  "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, t;\n\t"
+template <uint32_t BSTEP>
+__device__ __forceinline__ void mma8_tmem_a_run_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b0, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred e, t;\n\t.reg .b64 b;\n\t.reg .b32 a;\n\t"
+      "setp.eq.b32 t, %3, %3;\n\t"
+      "mov.b32 a, %1;\n\t"
+      "mov.b64 b, %2;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, t;\n\t" GDN_MMA_TA_NEXT GDN_MMA_TA_NEXT GDN_MMA_TA_NEXT
+          GDN_MMA_TA_NEXT GDN_MMA_TA_NEXT GDN_MMA_TA_NEXT GDN_MMA_TA_NEXT "}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b0), "r"(idesc), "n"(BSTEP)
+      : "memory");
+}
+#undef GDN_MMA_TA_NEXT
+
 // Byte offset of element (row, col) in a K-major 128B-swizzled operand
 // (64-element atom columns `acs` bytes apart). col % 8 == 0 addresses a chunk.
 __device__ __forceinline__ uint32_t sw128_off(int row, int col, uint32_t acs) {
