@@ -883,6 +883,12 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       float* vGf = vRho + 64;                               // G_r
       float* Ad = reinterpret_cast<float*>(sm + L::kAd);
 
+      // D's blocks off the diagonal are zero for every item (no other stage writes D)
+      for (int e = tid; e < 64 * 6; e += kCompute) {
+        const int row = e / 6, idx = e - row * 6, blk = row >> 4;
+        const int cc = idx < 2 * blk ? idx : idx + 2;
+        st_shared_v4(sbase + L::kDm + sw128_off(row, 8 * cc, 0), make_uint4(0, 0, 0, 0));
+      }
       for (int it = 0; !abort; ++it) {
         const int b = it & 1;
         const uint32_t* qe = reinterpret_cast<const uint32_t*>(sm + L::kQueue + b * L::kQueueBytes);
@@ -979,11 +985,9 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
 
         // ---- A (diagonal blocks fp32, off-diagonal blocks T) and P ----
         {
-          float gram[32];
-          tmem_ld32(tmem + tlane + kColG + 32 * ch, gram);
           const int rr = r128 & 63;
           const float Gr = vGf[rr];
-          float ck[32];   // this thread's 32 columns of vCk, in 16-byte loads
+          float ck[32];   // this thread's 32 columns of vCk, in 16-byte loads (before the TMEM load)
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const float4 t4 = reinterpret_cast<const float4*>(vCk + 32 * ch)[i];
@@ -992,6 +996,8 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             ck[4 * i + 2] = t4.z;
             ck[4 * i + 3] = t4.w;
           }
+          float gram[32];
+          tmem_ld32(tmem + tlane + kColG + 32 * ch, gram);
           float x[32];
           if (qd < 2) {
             const float fr = vB[rr] * vRk[rr] * (fast ? expf(Gr - gm) : 1.f);
@@ -1008,6 +1014,9 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
                 x[q2] = (sidx < rr) ? fr * ck[q2] * expf(Gr - vGf[sidx]) * gram[q2] : 0.f;
               }
             }
+            // the row's diagonal block (columns 16 blk .. 16 blk + 15) goes to A_d in fp32 and
+            // is zeroed in A_o; it lies in this thread's 32 columns when blk / 2 == ch (the
+            // columns left of it are kept, those right of it are already zero)
             const int blk = rr >> 4;
             if ((blk >> 1) == ch) {
               float4* dst = reinterpret_cast<float4*>(Ad + (blk * 16 + (rr & 15)) * L::kAdRow);
@@ -1015,14 +1024,16 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4)
                   dst[q4] = make_float4(x[16 + 4 * q4], x[17 + 4 * q4], x[18 + 4 * q4], x[19 + 4 * q4]);
+#pragma unroll
+                for (int q2 = 16; q2 < 32; ++q2) x[q2] = 0.f;
               } else {
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4)
                   dst[q4] = make_float4(x[4 * q4], x[1 + 4 * q4], x[2 + 4 * q4], x[3 + 4 * q4]);
+#pragma unroll
+                for (int q2 = 0; q2 < 16; ++q2) x[q2] = 0.f;
               }
             }
-#pragma unroll
-            for (int q2 = 0; q2 < 32; ++q2) x[q2] = (32 * ch + q2 < 16 * blk) ? x[q2] : 0.f;
 #pragma unroll
             for (int c8 = 0; c8 < 4; ++c8)
               st_shared_v4(sbase + L::kAo + sw128_off(rr, 32 * ch + 8 * c8, 0), pack8<T>(x + 8 * c8));
@@ -1046,11 +1057,13 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
               st_shared_v4(sbase + L::kPm + sw128_off(rr, 32 * ch + 8 * c8, 0), pack8<T>(x + 8 * c8));
           }
         }
-        cbar();
 
-        // ---- D = (I + A_d)^-1 ----
-        if (tid < 64) {
-          const int blk = tid >> 4, jj = tid & 15;
+        // ---- D = (I + A_d)^-1, by the two warps that wrote A_d's blocks (warp 0 blocks 0-1,
+        //      warp 5 blocks 2-3: row 16 blk + i of block blk is lane 16 (blk & 1) + i's);
+        //      D's other blocks are zero from before the first item ----
+        if (warp == 0 || warp == 5) {
+          __syncwarp();
+          const int blk = (warp == 5 ? 2 : 0) + (lane >> 4), jj = lane & 15;
           const float* Ab = Ad + blk * 16 * L::kAdRow;
           float xs[16];
 #pragma unroll
@@ -1067,12 +1080,6 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
 #pragma unroll
           for (int i = 0; i < 16; ++i)
             st_shared_u16(sbase + L::kDm + sw128_off(16 * blk + i, 16 * blk + jj, 0), Op16<T>::one(xs[i]));
-        } else {
-          for (int e = tid - 64; e < 64 * 6; e += kCompute - 64) {
-            const int row = e / 6, idx = e - row * 6, blk = row >> 4;
-            const int cc = idx < 2 * blk ? idx : idx + 2;
-            st_shared_v4(sbase + L::kDm + sw128_off(row, 8 * cc, 0), make_uint4(0, 0, 0, 0));
-          }
         }
         publish(true);
 
