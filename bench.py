@@ -74,7 +74,8 @@ def decode_bytes(B, Hqk, Hv, d, state_bytes=4):
 
 # the source files each kernel is built from (its traffic record is void once one changes)
 KERNEL_SOURCES = {
-    "prefill_pc": ("common.cuh", "sm100.cuh", "prefill_pc.cuh"),
+    "prefill_pc": ("common.cuh", "sm100.cuh", "prefill_pc.cuh"),        # 32-row slices, 4096 tokens
+    "prefill_pc_long": ("common.cuh", "sm100.cuh", "prefill_pc.cuh"),   # 128-row slices, 32768 tokens
     "decode": ("common.cuh", "decode.cuh"),
 }
 
@@ -100,6 +101,8 @@ def kernel_source_hash(kernel):
 def traffic_record(kernel):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
     the current kernel source; else None."""
+    if kernel not in KERNEL_SOURCES:
+        return None
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
@@ -459,13 +462,14 @@ def workload_config(w, copies=None, n=1):
     return cfg
 
 
-def prefill_subline(r, w, steps, ms_max, world, pk, pk_kind):
-    """A prefill workload's sub-object of the JSON line."""
+def prefill_subline(r, w, steps, ms_max, world, pk, pk_kind, traffic=None):
+    """A prefill workload's sub-object of the JSON line (traffic: DRAM bytes per
+    launch from an ncu capture, or None)."""
     fl = prefill_flops_per_token_head(w.chunk, w.d) * r["tokens"] * w.Hv
     return {"value": aggregate_rate(r["tokens"], ms_max, world), "unit": "tokens/s", "ms_per_step": ms_max,
             "steps": steps, "timed_replays": r["replays"], "gpu_launches": steps,
             "config": workload_config(w, r["copies"], world),
-            "roofline": roofline_tensor(fl, r["ms"], pk, pk_kind),
+            "roofline": roofline_tensor(fl, r["ms"], pk, pk_kind, traffic=traffic),
             "roofline_hbm_view": roofline_hbm(r["bytes"], r["ms"], pk, pk_kind),
             "binding_frac": binding_frac(fl, r["bytes"], r["ms"], pk)}
 
@@ -579,7 +583,9 @@ def main():
         ms = max_over_ranks(r["ms"])
         value = aggregate_rate(r["tokens"], ms, world)
         flops = prefill_flops_per_token_head(w.chunk, w.d) * r["tokens"] * w.Hv
-        tr = traffic_record("prefill_pc")
+        # the ncu captures were taken on the 4096-token layer and on the 32768-token prompt
+        tr = traffic_record({"prefill": "prefill_pc", "long": "prefill_pc_long"}.get(w.name, "")) \
+            if w.total_tokens in (4096, 32768) else None
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": DATA,
@@ -641,13 +647,20 @@ def main():
         del rl["graph"]
         msl = max_over_ranks(rl["ms"])
         fl = prefill_flops_per_token_head(wl.chunk, wl.d) * rl["tokens"] * wl.Hv
-        line["long_prefill"] = prefill_subline(rl, wl, nl, msl, world, pk, pk_kind)
+        trl = traffic_record("prefill_pc_long")   # captured on this workload itself
+        line["long_prefill"] = prefill_subline(rl, wl, nl, msl, world, pk, pk_kind,
+                                               traffic=trl["bytes_per_launch"] if trl else None)
         # the longest prompt: 81920 tokens, 16 q/k and 32 v heads
         wx = workloads.workload("long", T=81920)
         nx = max(2, args.steps // 10)
         rx = run_prefill_bench(gdn, wx, nx, args.warmup, device, rank)
         del rx["graph"]
-        line["long_prefill_81920"] = prefill_subline(rx, wx, nx, max_over_ranks(rx["ms"]), world, pk, pk_kind)
+        # (the 32768-token capture scaled by the tokens: every (head, chunk) moves the same bytes)
+        line["long_prefill_81920"] = prefill_subline(
+            rx, wx, nx, max_over_ranks(rx["ms"]), world, pk, pk_kind,
+            traffic=round(trl["bytes_per_launch"] * wx.total_tokens / wl.total_tokens) if trl else None)
+        if trl:
+            line["long_prefill_81920"]["roofline"]["traffic_scaled_from"] = "the 32768-token capture, by tokens"
         # packed varlen: 8 sequences of 128..8192 tokens with their own states
         wv = workloads.workload("varlen")
         nv = max(2, args.steps // 4)
