@@ -629,9 +629,12 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             // the buffer (no CTA-wide barrier here)
             fence_async_smem();
             tc_fence_before();
-            if constexpr (DVP >= 64) {   // the state-written arrival does not wait for the O tile's read
-              __syncwarp();              // (measured side by side on the B200: 0.6-0.8 % faster at
-              if (lane == 0 && c + 1 < nch) mbar_arrive(bar_s);   // 128-row slices, 0.5 % slower at 32)
+            // At 64-row slices and wider the state-written arrival does not wait for the O
+            // tile's read (measured side by side on the B200: 0.6-0.8 % faster at 128-row
+            // slices, 0.5 % slower at 32).
+            if constexpr (DVP >= 64) {
+              __syncwarp();
+              if (lane == 0 && c + 1 < nch) mbar_arrive(bar_s);
               if (tid == 64) bulk_wait_read_all();   // the O tile has left the buffer
               __syncwarp();
               if (lane == 0) mbar_arrive(&bar_free[b]);
