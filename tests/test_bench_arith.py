@@ -56,3 +56,34 @@ def test_roofline_fractions():
 def test_aggregate_rate_counts_every_rank_at_the_slowest_time():
     assert bench.aggregate_rate(4096, 0.1, 1) == pytest.approx(40.96e6)
     assert bench.aggregate_rate(4096, 0.1, 8) == pytest.approx(8 * 40.96e6)
+
+
+def test_traffic_records_are_keyed_by_kernel_source():
+    """Each committed ncu traffic record names the kernel source it was taken on:
+    it is served while that source is unchanged (comments aside) and dropped
+    once the code differs; an unknown kernel has no record."""
+    import json
+    import os
+    with open(os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
+        recs = json.load(f)
+    for kernel in ("prefill_pc", "prefill_pc_long", "decode"):
+        assert kernel in recs and kernel in bench.KERNEL_SOURCES
+        rec = recs[kernel]
+        assert rec["bytes_per_launch"] == rec["dram_read_bytes"] + rec["dram_write_bytes"]
+        current = rec["source_hash"] == bench.kernel_source_hash(kernel)
+        assert bench.traffic_record(kernel) == (rec if current else None)
+    assert bench.traffic_record("no_such_kernel") is None
+    src = "int a = 1; // note\n/* block */ int b = 2;"
+    assert bench._code_only(src) == bench._code_only(src.replace("note", "other note"))
+    assert bench._code_only(src) != bench._code_only(src.replace("b = 2", "b = 3"))
+
+
+def test_long_prompt_traffic_stays_below_its_algorithmic_bytes():
+    """The 32768-token capture's DRAM bytes are at most the prompt's algorithmic
+    bytes (inputs once, outputs once): the package ring stays in L2."""
+    import json
+    import os
+    with open(os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
+        rec = json.load(f)["prefill_pc_long"]
+    alg = bench.prefill_bytes(32768, 16, 32, 128, 1, True)
+    assert rec["bytes_per_launch"] <= alg
