@@ -81,8 +81,8 @@ struct DecodeShape {
   static constexpr int kRowsPerSlot = 32 / kLanesPerRow;
   // 4 fp32 rows or 16 bf16 rows per warp: at d_k = 128 every lane keeps 4 (fp32) or 8
   // (bf16) independent 16-byte loads in flight (measured on B200 at 64 sequences x 32
-  // heads: 4 fp32 rows 47.2 us a step against 49.1 with 8 and 70 with 2; 16 bf16 rows
-  // 30.1 against 31.7 with 8)
+  // heads: 4 fp32 rows 47.2 us a step against 49.1 with 8 and 70 with 2, and 47.4 against
+  // 49.4 with 3, 47.9 with 5 and 47.6 with 6; 16 bf16 rows 30.1 against 31.7 with 8)
   static constexpr int kRowsTarget = sizeof(TS) == 4 ? 4 : 16;
   static constexpr int kSlots = kRowsTarget / kRowsPerSlot > 0 ? kRowsTarget / kRowsPerSlot : 1;
   static constexpr int kRowsPerWarp = kRowsPerSlot * kSlots;
